@@ -1,0 +1,161 @@
+"""CPU oracle for paged decode attention, reshape_and_cache and copy_blocks.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library (``paged_kv_cache_424_b200``) and never imports it.
+
+The arithmetic lives in ``pa_oracle.c`` (plain C, double precision, OpenMP over
+(sequence, head) pairs), built into ``liboracle.so`` by :func:`build`.  This
+module only marshals numpy arrays into it.  ``brute.py`` holds a pure-Python
+restatement for tiny inputs.
+
+Every function below states what it computes; the C source cites the pages.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F16 = 0
+BF16 = 1
+_DTYPE_CODE = {"f16": F16, "fp16": F16, "float16": F16, "bf16": BF16, "bfloat16": BF16}
+
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB, extra: Sequence[str] = ()) -> str:
+    """Compile the C oracle with gcc into a shared library and return its path."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", *extra, "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _stale(lib: str, src: str) -> bool:
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+def load(path: str | None = None):
+    """Load (building first if missing or stale) and return an :class:`Oracle`."""
+    global _lib
+    if path is not None:
+        return Oracle(path)
+    if _lib is None:
+        if _stale(_LIB, _SRC):
+            build()
+        _lib = Oracle(_LIB)
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+class Oracle:
+    """ctypes handle on one build of ``pa_oracle.c``."""
+
+    def __init__(self, path: str):
+        self.path = path
+        lib = ctypes.CDLL(path)
+        vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        lib.oracle_paged_decode.argtypes = [vp, vp, vp, vp, vp, vp, dbl, i32, i32, i32, i32, i32, i32, i64, i32]
+        lib.oracle_paged_decode.restype = ctypes.c_int
+        lib.oracle_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64]
+        lib.oracle_reshape_and_cache.restype = ctypes.c_int
+        lib.oracle_copy_blocks.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, i64]
+        lib.oracle_copy_blocks.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.restype = ctypes.c_int
+        self._lib = lib
+
+    # -- threads ---------------------------------------------------------
+    def set_num_threads(self, n: int) -> int:
+        return int(self._lib.oracle_set_num_threads(int(n)))
+
+    def max_threads(self) -> int:
+        return int(self._lib.oracle_max_threads())
+
+    # -- operations ------------------------------------------------------
+    def paged_decode(self, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                     dtype: str) -> np.ndarray:
+        """out[s, h, :] = softmax(scale * q[s,h] . K_s^T) V_s, in float64.
+
+        ``q`` is ``[S, H, D]`` and the caches ``[NB, Hk, B, D]``, all uint16
+        bit patterns of ``dtype``; K_s / V_s are gathered through
+        ``block_tables`` (``[S, MB]`` int32) for the first ``context_lens[s]``
+        positions.
+        """
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        k_cache = np.ascontiguousarray(k_cache, dtype=np.uint16)
+        v_cache = np.ascontiguousarray(v_cache, dtype=np.uint16)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, H, D = q.shape
+        NB, Hk, B, D2 = k_cache.shape
+        if D2 != D or v_cache.shape != k_cache.shape or bt.shape[0] != S or cl.shape != (S,):
+            raise OracleError("shape mismatch")
+        MB = bt.shape[1] if bt.ndim == 2 else 0
+        out = np.zeros((S, H, D), dtype=np.float64)
+        rc = self._lib.oracle_paged_decode(_p(out), _p(q), _p(k_cache), _p(v_cache), _p(bt), _p(cl),
+                                           float(scale), S, H, Hk, D, B, MB, NB, _DTYPE_CODE[dtype])
+        if rc != 0:
+            raise OracleError(f"oracle_paged_decode returned {rc}")
+        return out
+
+    def reshape_and_cache(self, k_cache, v_cache, key, value, slot_mapping) -> None:
+        """In place: k_cache[slot // B, :, slot % B, :] = key[t] for slot >= 0."""
+        for a in (k_cache, v_cache):
+            if a.dtype != np.uint16 or not a.flags.c_contiguous:
+                raise OracleError("caches must be C-contiguous uint16")
+        key = np.ascontiguousarray(key, dtype=np.uint16)
+        value = np.ascontiguousarray(value, dtype=np.uint16)
+        sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        NB, Hk, B, D = k_cache.shape
+        T = sm.shape[0]
+        if key.shape != (T, Hk, D) or value.shape != (T, Hk, D):
+            raise OracleError("key/value shape mismatch")
+        rc = self._lib.oracle_reshape_and_cache(_p(k_cache), _p(v_cache), _p(key), _p(value), _p(sm),
+                                                T, Hk, D, B, NB)
+        if rc != 0:
+            raise OracleError(f"oracle_reshape_and_cache returned {rc}")
+
+    def copy_blocks(self, k_caches, v_caches, block_mapping) -> None:
+        """In place, per layer: block dst of K and V becomes a copy of block src."""
+        bm = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+        L = len(k_caches)
+        if L != len(v_caches) or L == 0:
+            raise OracleError("need matching non-empty K and V cache lists")
+        NB, Hk, B, D = k_caches[0].shape
+        for a in list(k_caches) + list(v_caches):
+            if a.shape != (NB, Hk, B, D) or a.dtype != np.uint16 or not a.flags.c_contiguous:
+                raise OracleError("every cache must be C-contiguous uint16 of one shape")
+        kp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in k_caches])
+        vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_caches])
+        rc = self._lib.oracle_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
+                                          L, _p(bm), bm.shape[0], Hk, D, B, NB)
+        if rc != 0:
+            raise OracleError(f"oracle_copy_blocks returned {rc}")
+
+
+def paged_decode(*args, **kw):
+    return load().paged_decode(*args, **kw)
+
+
+def reshape_and_cache(*args, **kw):
+    return load().reshape_and_cache(*args, **kw)
+
+
+def copy_blocks(*args, **kw):
+    return load().copy_blocks(*args, **kw)

@@ -1,0 +1,257 @@
+/*
+ * pa_oracle.c -- plain, slow, double-precision CPU oracle for paged decode
+ * attention and its two companion cache operations.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the package smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library; the two meet only at the documented memory layouts.
+ *
+ * What it follows (sources are the web pages this library is built from):
+ *  - "vLLM PagedAttention 大模型推理架构深度实战" (ybb.press), section 2.2
+ *    "PagedAttention核心机制": the KV cache is cut into fixed blocks of 16
+ *    tokens; each sequence owns a block table that maps its logical block
+ *    index to a physical block, like an OS page table.
+ *  - "vLLM：重塑大模型推理性能的关键引擎" (unionyoga.cn), section
+ *    "vLLM 如何破局？从PagedAttention说起", kernel sketch: a sequence needs
+ *    ceil(context_len / BLOCK_SIZE) blocks; logical block i of sequence s is
+ *    block_table[s * MAX_BLOCKS + i].
+ *  - The same ybb.press page, section 2.1 and section 5.1: decode attention
+ *    of a new token against all cached keys/values is exact attention,
+ *    softmax(q K^T * scale) V.  No approximation is involved, so this oracle
+ *    is that definition written out (two-pass, max-subtracted softmax, which
+ *    is the same function), not the online/blocked algorithm the GPU runs.
+ *  - ybb.press section 2.3 "写时复制与并行采样": a shared block is copied
+ *    before a sharer modifies it; copy_blocks is a plain byte copy.
+ *  - ybb.press section 六 "架构总览" (decode loop): each iteration writes the
+ *    new token's K/V into its KV-cache block; reshape_and_cache is the plain
+ *    indexed assignment.
+ *
+ * Layouts (row-major, contiguous; element = 16-bit fp16 or bf16 bit pattern):
+ *   q, out        [num_seqs, num_heads, head_dim]   (out is double here)
+ *   k/v cache     [num_blocks, num_kv_heads, block_size, head_dim]
+ *   block_tables  [num_seqs, max_blocks_per_seq] int32
+ *   context_lens  [num_seqs] int32
+ *   key/value     [num_tokens, num_kv_heads, head_dim]
+ *   slot_mapping  [num_tokens] int64, slot = block * block_size + offset,
+ *                 negative = skip
+ *   block_mapping [num_pairs, 2] int64 (src, dst)
+ *
+ * Readings where the pages are silent: query head h reads KV head
+ * h / (num_heads / num_kv_heads) (contiguous GQA groups); a context length of
+ * zero yields an all-zero output row.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_ARG (-1)
+#define ORC_ERR_RANGE (-2)
+#define ORC_ERR_NOMEM (-3)
+
+#define ORC_F16 0
+#define ORC_BF16 1
+
+/* IEEE 754 binary16 -> double, exactly: sign, 5-bit exponent (bias 15),
+ * 10-bit fraction; exponent 0 is subnormal (fraction * 2^-24). */
+static double widen_f16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m + 1024), e - 25);
+    return sign ? -v : v;
+}
+
+/* bfloat16 is the top half of an IEEE binary32: put it back and widen. */
+static double widen_bf16(uint16_t h) {
+    uint32_t bits = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static double widen(uint16_t h, int32_t dtype) {
+    return dtype == ORC_BF16 ? widen_bf16(h) : widen_f16(h);
+}
+
+int oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Decode attention for every (sequence, query head).
+ *
+ * For sequence s with n = context_lens[s] tokens and query head h
+ * (KV head kvh = h / group):
+ *   K_s[j] = k_cache[block_tables[s, j / block_size], kvh, j % block_size, :]
+ *   x_j    = scale * sum_d q[s, h, d] * K_s[j, d]                (j < n)
+ *   out[s, h, :] = sum_j softmax(x)_j * V_s[j, :]
+ * Only slots j < n are read: the tail of the last block and the table
+ * entries past ceil(n / block_size) are never touched.
+ */
+int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache,
+                        const uint16_t *v_cache, const int32_t *block_tables,
+                        const int32_t *context_lens, double scale, int32_t num_seqs,
+                        int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t block_size, int32_t max_blocks_per_seq,
+                        int64_t num_blocks, int32_t dtype) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return ORC_ERR_ARG;
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_blocks_per_seq < 0 || num_blocks <= 0)
+        return ORC_ERR_ARG;
+    if (num_heads % num_kv_heads != 0) return ORC_ERR_ARG;
+    if (dtype != ORC_F16 && dtype != ORC_BF16) return ORC_ERR_ARG;
+
+    /* Every referenced block id must lie in the pool. */
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t n = context_lens[s];
+        if (n < 0 || (int64_t)n > (int64_t)max_blocks_per_seq * block_size) return ORC_ERR_RANGE;
+        int32_t nblk = (n + block_size - 1) / block_size;
+        for (int32_t i = 0; i < nblk; ++i) {
+            int32_t b = block_tables[(int64_t)s * max_blocks_per_seq + i];
+            if (b < 0 || (int64_t)b >= num_blocks) return ORC_ERR_RANGE;
+        }
+    }
+
+    const int32_t group = num_heads / num_kv_heads;
+    const int64_t pairs = (int64_t)num_seqs * num_heads;
+    int status = ORC_OK;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < pairs; ++p) {
+        const int32_t s = (int32_t)(p / num_heads);
+        const int32_t h = (int32_t)(p % num_heads);
+        const int32_t kvh = h / group;
+        const int32_t n = context_lens[s];
+        double *o = out + p * head_dim;
+        for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+        if (n == 0) continue;
+
+        double *x = (double *)malloc(sizeof(double) * (size_t)n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        if (!x || !qd) {
+            free(x);
+            free(qd);
+#pragma omp atomic write
+            status = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int32_t d = 0; d < head_dim; ++d) qd[d] = widen(q[p * head_dim + d], dtype);
+
+        /* Pass 1: logits through the block table. */
+        for (int32_t j = 0; j < n; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double dot = 0.0;
+            for (int32_t d = 0; d < head_dim; ++d) dot += qd[d] * widen(k_cache[row + d], dtype);
+            x[j] = scale * dot;
+        }
+        /* Softmax: subtract the max (the result is unchanged), normalise. */
+        double m = x[0];
+        for (int32_t j = 1; j < n; ++j)
+            if (x[j] > m) m = x[j];
+        double z = 0.0;
+        for (int32_t j = 0; j < n; ++j) {
+            x[j] = exp(x[j] - m);
+            z += x[j];
+        }
+        /* Pass 2: probability-weighted sum of the values. */
+        for (int32_t j = 0; j < n; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double w = x[j] / z;
+            for (int32_t d = 0; d < head_dim; ++d) o[d] += w * widen(v_cache[row + d], dtype);
+        }
+        free(x);
+        free(qd);
+    }
+    return status;
+}
+
+/*
+ * Cache write: for every token t with slot = slot_mapping[t] >= 0,
+ *   k_cache[slot / block_size, h, slot % block_size, :] = key[t, h, :]
+ * and the same for value, for every KV head h.  Tokens are applied in order.
+ */
+int oracle_reshape_and_cache(uint16_t *k_cache, uint16_t *v_cache, const uint16_t *key,
+                             const uint16_t *value, const int64_t *slot_mapping,
+                             int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                             int32_t block_size, int64_t num_blocks) {
+    if (!k_cache || !v_cache || (num_tokens > 0 && (!key || !value || !slot_mapping)))
+        return ORC_ERR_ARG;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return ORC_ERR_ARG;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot / block_size >= num_blocks) return ORC_ERR_RANGE;
+    }
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                k_cache[dst + d] = key[src + d];
+                v_cache[dst + d] = value[src + d];
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/*
+ * Copy-on-write duplication: for every layer and every pair (src, dst),
+ * copy all num_kv_heads * block_size * head_dim elements of block src to
+ * block dst, in the K and the V cache.  Pairs are applied in order.
+ */
+int oracle_copy_blocks(uint16_t *const *k_caches, uint16_t *const *v_caches, int32_t num_layers,
+                       const int64_t *block_mapping, int32_t num_pairs, int32_t num_kv_heads,
+                       int32_t head_dim, int32_t block_size, int64_t num_blocks) {
+    if (num_layers < 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_blocks <= 0)
+        return ORC_ERR_ARG;
+    if ((num_layers > 0 && (!k_caches || !v_caches)) || (num_pairs > 0 && !block_mapping))
+        return ORC_ERR_ARG;
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return ORC_ERR_RANGE;
+    }
+    const int64_t elems = (int64_t)num_kv_heads * block_size * head_dim;
+    for (int32_t l = 0; l < num_layers; ++l) {
+        if (!k_caches[l] || !v_caches[l]) return ORC_ERR_ARG;
+        for (int32_t i = 0; i < num_pairs; ++i) {
+            int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
+            memmove(k_caches[l] + dst * elems, k_caches[l] + src * elems, sizeof(uint16_t) * elems);
+            memmove(v_caches[l] + dst * elems, v_caches[l] + src * elems, sizeof(uint16_t) * elems);
+        }
+    }
+    return ORC_OK;
+}

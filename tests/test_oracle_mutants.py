@@ -1,0 +1,69 @@
+"""Every plausible mistake planted in the oracle must fail at least one pin.
+
+Each mutant is a copy of ``oracle/pa_oracle.c`` with one textual change
+(a dropped term, a wrong sign, a wrong index or layout, a transposed
+operand), compiled with gcc into a temporary library and run against the pin
+suite.  A mutant that passes every pin would mean the pins cannot tell that
+mistake from the correct oracle.  Only the CPU oracle is mutated.
+"""
+import os
+
+import pytest
+
+import oracle
+from pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
+
+ROW = "((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim"
+MUTANTS = {
+    "drop_scale": ("x[j] = scale * dot;", "x[j] = dot;"),
+    "gqa_head_map": ("const int32_t kvh = h / group;", "const int32_t kvh = h % num_kv_heads;"),
+    "table_index_shift": ("block_tables[(int64_t)s * max_blocks_per_seq + j / block_size]",
+                          "block_tables[(int64_t)s * max_blocks_per_seq + (j / block_size + 1) % "
+                          "max_blocks_per_seq]"),
+    "token_major_layout": (ROW, "((blk * block_size + j % block_size) * num_kv_heads + kvh) * head_dim"),
+    "no_max_subtraction": ("x[j] = exp(x[j] - m);", "x[j] = exp(x[j]);"),
+    "exp_sign": ("x[j] = exp(x[j] - m);", "x[j] = exp(m - x[j]);"),
+    "normalise_by_length": ("double w = x[j] / z;", "double w = x[j] / n;"),
+    "read_past_length": ("const int32_t n = context_lens[s];",
+                         "const int32_t n = context_lens[s] + (context_lens[s] % block_size != 0);"),
+    "f16_exponent_bias": ("e - 25);", "e - 24);"),
+    "f16_subnormal_scale": ("ldexp((double)m, -24)", "ldexp((double)m, -25)"),
+    "bf16_shift": ("(uint32_t)h << 16;", "(uint32_t)h << 15;"),
+    "values_from_key_cache": ("o[d] += w * widen(v_cache[row + d], dtype);",
+                              "o[d] += w * widen(k_cache[row + d], dtype);"),
+    "query_head_zero": ("qd[d] = widen(q[p * head_dim + d], dtype);",
+                        "qd[d] = widen(q[(p - h) * head_dim + d], dtype);"),
+    "max_not_updated": ("if (x[j] > m) m = x[j];", "if (x[j] < m) m = x[j];"),
+    "write_slot_shift": ("int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;",
+                         "int64_t dst = ((blk * num_kv_heads + h) * block_size + (off + 1) % block_size)"
+                         " * head_dim;"),
+    "write_key_into_value": ("v_cache[dst + d] = value[src + d];", "v_cache[dst + d] = key[src + d];"),
+    "copy_only_k": ("memmove(v_caches[l] + dst * elems, v_caches[l] + src * elems, sizeof(uint16_t) * elems);",
+                    ""),
+    "copy_reversed": ("memmove(k_caches[l] + dst * elems, k_caches[l] + src * elems",
+                      "memmove(k_caches[l] + src * elems, k_caches[l] + dst * elems"),
+    "zero_length_not_zeroed": ("for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;\n        if (n == 0) continue;",
+                               "if (n == 0) { o[0] = 1.0; continue; }\n        "
+                               "for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert old in src, f"mutant {name}: pattern no longer in the oracle source"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.build(str(path), str(tmp_path / "libmutant.so"))
+    orc = oracle.load(lib)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, oracle.OracleError) as e:  # noqa: PERF203
+            failed.append(pin.__name__)
+            break
+    assert failed, f"mutant {name} passed every pin"
