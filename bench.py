@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark: paged decode attention on B200, one JSON line on stdout.
+
+A step is one pass of the whole hot path over one batch: the cache write of
+every sequence's new token (pa_reshape_and_cache), copy-on-write copies when
+the workload has them (pa_copy_blocks), and decode attention of every
+sequence over its paged KV cache (pa_decode, with the split-KV merge when a
+context spans several 512-token partitions).  Default workload: the
+Llama-2-7B-shaped MHA batch (64 sequences, lengths U[128, 2048], 32 heads,
+head_dim 128, fp16, 16384-block pool).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...      # the CPU oracle, timed the same way
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of
+the same shape (sequences are independent; no collective on the data path),
+so per-GPU work is fixed: weak scaling.  Timing is CUDA events on the
+launching stream, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention seqs/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha7b", choices=["tiny", "mha7b", "gqa8b", "long70b", "cow"])
+    ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
+    ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
+    ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    return ap.parse_args(argv)
+
+
+def make_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
+    from paged_kv_cache_424_b200 import workload as W
+    kw = {}
+    if num_seqs is not None:
+        kw["num_seqs"] = num_seqs
+    if num_blocks is not None:
+        kw["num_blocks"] = num_blocks
+    if name == "tiny":
+        return W.tiny(seed)
+    if name == "cow":
+        if num_seqs is not None:
+            kw = {"num_prompts": max(1, num_seqs // 8), **({"num_blocks": num_blocks} if num_blocks else {})}
+        return W.cow(seed, **kw)
+    return getattr(W, name)(seed, **kw)
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_424_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, units: float):
+    """DRAM bytes per decode launch from the committed ncu summary, scaled to
+    this launch's units, or None if absent or taken on other kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_src_sha") != kernel_source_hash():
+        return None
+    ent = rec.get("workloads", {}).get(workload)
+    if not ent:
+        return None
+    return float(ent["dram_bytes_per_unit"]) * units
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"NVML unavailable: {self.err}"}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def cpu_baseline(sc, seconds: float):
+    """The oracle as it stands on this host's cores, on repeated full steps of
+    the workload (or a subset of its sequences when one step is too long)."""
+    import oracle
+    from oracle.harness import OracleSession
+    orc = oracle.load()
+    cores = orc.max_threads()
+    st = sc.steps[0]
+    ses = OracleSession(sc, oracle=orc)
+    ses.apply_cache_ops(st)          # admission + writes, outside the timing
+    S = sc.dims.num_seqs
+    t0 = time.perf_counter()
+    ses.decode(st, np.arange(min(S, 4)))
+    t_seq = (time.perf_counter() - t0) / min(S, 4)
+    n = int(max(1, min(S, seconds / max(t_seq, 1e-9))))
+    seqs_done, t_total, reps = 0, 0.0, 0
+    while t_total < seconds or reps == 0:
+        sel = (np.arange(n) + reps * n) % S
+        t0 = time.perf_counter()
+        for w in st.writes:   # the step's cache write, on the host pool
+            sm = ses.pool.relabel_slots(w.slot_mapping, sc.dims.block_size)
+            k, v = ses.pool.view()
+            orc.reshape_and_cache(k, v, w.key, w.value, sm)
+        ses.decode(st, sel)
+        t_total += time.perf_counter() - t0
+        seqs_done += n
+        reps += 1
+        if t_total > 3 * seconds:
+            break
+    return {"value": seqs_done / t_total, "unit": "seqs/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x ({n} of {S} sequences: cache write of the step + float64 decode), "
+                      f"{t_total:.1f} s, {cores} OpenMP threads"}
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup(args)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    from paged_kv_cache_424_b200 import build
+    build.build()
+    from paged_kv_cache_424_b200 import binding as pa
+    from paged_kv_cache_424_b200 import workload as W
+    from paged_kv_cache_424_b200.session import DeviceSession, to_device
+
+    sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks)
+    st = sc.steps[0]
+    d = sc.dims
+    P = sc.partition_tokens if args.partition is None else args.partition
+    dev = DeviceSession(sc, device=str(device))
+    dev.apply_cache_ops(st)                      # prefill admission + first writes (untimed set-up)
+    inp = dev.decode_inputs(st)
+    writes = dev.write_inputs(st)
+    bm = torch.from_numpy(np.ascontiguousarray(st.block_mapping)).to(device) if st.block_mapping.size else None
+    maxlen = st.max_context_len
+    dims = pa.dims_of(inp["q"], dev.k_cache, inp["block_tables"])
+    nparts = pa.pa_decode_num_partitions(dims, maxlen, P)
+    ws = dev.workspace(pa.pa_decode_workspace_size(dims, maxlen, P))
+    out = torch.empty((d.num_seqs, d.num_heads, d.head_dim), dtype=dev.dtype, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(e0=None, e1=None):
+        if bm is not None:
+            pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], bm, stream=stream)
+        for key, value, slots in writes:
+            pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
+        if e0 is not None:
+            e0.record(stream)
+        pa.pa_decode(out, inp["q"], dev.k_cache, dev.v_cache, inp["block_tables"], inp["context_lens"], sc.scale,
+                     d.num_kv_heads, maxlen, P, ws, stream=stream)
+        if e1 is not None:
+            e1.record(stream)
+
+    launches_per_step = (1 if bm is not None else 0) + len(writes) + (2 if nparts > 1 else 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if pa.pa_device_error(stream) != 0:
+        raise SystemExit("device error word set during warm-up")
+
+    K = args.steps
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        start.record(stream)
+        for i in range(K):
+            step(e0[i], e1[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world)
+    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
+    dec_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
+    dec_avg_ms = max_over_ranks(sum(dec_ms) / K, world, device)
+
+    # ---- end to end: host buffers in, result out, through the same calls ----
+    e2e = None
+    if not args.no_e2e:
+        h_q = inp["q"].cpu().pin_memory()
+        h_bt = inp["block_tables"].cpu().pin_memory()
+        h_cl = inp["context_lens"].cpu().pin_memory()
+        h_w = [(k.cpu().pin_memory(), v.cpu().pin_memory(), s.cpu().pin_memory()) for k, v, s in writes]
+        h_bm = st.block_mapping
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        d_q, d_bt, d_cl = torch.empty_like(inp["q"]), torch.empty_like(inp["block_tables"]), torch.empty_like(
+            inp["context_lens"])
+        d_w = [(torch.empty_like(k), torch.empty_like(v), torch.empty_like(s)) for k, v, s in writes]
+        h_bm_t = torch.from_numpy(np.ascontiguousarray(h_bm)).pin_memory() if bm is not None else None
+        d_bm = torch.empty_like(bm) if bm is not None else None
+        h2d = (h_q.numel() * h_q.element_size() + h_bt.numel() * 4 + h_cl.numel() * 4 +
+               sum(k.numel() * k.element_size() * 2 + s.numel() * 8 for k, _, s in h_w) +
+               (h_bm_t.numel() * 8 if h_bm_t is not None else 0))
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            d_q.copy_(h_q, non_blocking=True)
+            d_bt.copy_(h_bt, non_blocking=True)
+            d_cl.copy_(h_cl, non_blocking=True)
+            for (hk, hv, hs), (dk, dv, ds) in zip(h_w, d_w):
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                ds.copy_(hs, non_blocking=True)
+            if d_bm is not None:
+                d_bm.copy_(h_bm_t, non_blocking=True)
+                pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], d_bm, stream=stream)
+            for dk, dv, ds in d_w:
+                pa.pa_reshape_and_cache(dk, dv, dev.k_cache, dev.v_cache, ds, stream=stream)
+            pa.pa_decode(out, d_q, dev.k_cache, dev.v_cache, d_bt, d_cl, sc.scale, d.num_kv_heads, maxlen, P, ws,
+                         stream=stream)
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(min(args.warmup, 10)):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        Ke = max(1, min(K, 500))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
+        e2e = {"value": d.num_seqs * Ke * world / (e2e_ms / 1e3), "unit": "seqs/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": Ke,
+               "path": "pinned host buffers -> cudaMemcpyAsync -> pa_* C-ABI calls -> output copied back"}
+
+    if pa.pa_device_error(stream) != 0:
+        raise SystemExit("device error word set during the timed region")
+
+    kv = W.kv_bytes(st, d)
+    algo = kv + W.qo_bytes(d)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = algo / (dec_avg_ms / 1e3) / 1e9
+    traffic = ncu_traffic(args.workload, units=float(st.context_lens.sum()))
+    result = {
+        "metric": METRIC,
+        "value": d.num_seqs * K * world / (ms_total / 1e3),
+        "unit": "seqs/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_total / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": d.dtype,
+        "data": "synthetic (seeded U[-1,1] fp16/bf16 values, NaN in every unused slot; no dataset)",
+        "config": {"workload": f"{sc.name}: {sc.note}", "global_batch": d.num_seqs * world,
+                   "seq_len": "per-sequence, " + f"mean {float(st.context_lens.mean()):.0f}, "
+                              f"max {int(st.context_lens.max())}",
+                   "partition_tokens": P, "num_partitions": nparts,
+                   "parallelism": f"{world} independent batches (one per GPU, no data-path collective)",
+                   "l2": f"inputs larger than L2: {kv / 1e9:.2f} GB of KV read per step vs 126 MB L2",
+                   "kv_bytes_per_step": kv, "algorithmic_bytes_per_step": algo},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "pa_decode (decode kernel + log-sum-exp merge)" if nparts > 1 else "pa_decode",
+                     "kernel_ms": dec_avg_ms, "frac_of_8000": achieved / 8000.0},
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(sc, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, timed like our arm
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import oracle
+    from oracle.harness import OracleSession
+    orc = oracle.load()
+    cores = orc.max_threads()
+    sc = make_scenario(args.workload, seed=1, num_seqs=args.num_seqs, num_blocks=args.num_blocks)
+    st = sc.steps[0]
+    S = sc.dims.num_seqs
+    ses = OracleSession(sc, oracle=orc)
+    ses.apply_cache_ops(st)
+    t0 = time.perf_counter()
+    ses.decode(st, np.arange(min(S, 2)))
+    t_seq = (time.perf_counter() - t0) / min(S, 2)
+    budget = 120.0 / max(1, args.steps + args.warmup)          # seconds per step
+    n = int(max(1, min(S, budget / max(t_seq, 1e-9))))
+
+    def one(i):
+        sel = (np.arange(n) + i * n) % S
+        for w in st.writes:
+            sm = ses.pool.relabel_slots(w.slot_mapping, sc.dims.block_size)
+            k, v = ses.pool.view()
+            orc.reshape_and_cache(k, v, w.key, w.value, sm)
+        ses.decode(st, sel)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = f"each step: {n} of {S} sequences (cache write + float64 decode), {cores} OpenMP threads"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{sc.name}: {sc.note}", "global_batch": S, "sample_seqs_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "seqs/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "seqs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,176 @@
+/*
+ * pa.h -- C ABI of the paged decode attention library (libpa.so, sm_100a).
+ *
+ * Three operations make one decode step of one attention layer over a KV
+ * cache stored in fixed 16-token physical blocks:
+ *
+ *   pa_reshape_and_cache  write each new token's key/value into its slot
+ *   pa_copy_blocks        copy-on-write duplication of shared blocks
+ *   pa_decode             single-query attention of every sequence over its
+ *                         cached tokens, gathered through its block table
+ *
+ * Sources: "vLLM PagedAttention 大模型推理架构深度实战" (ybb.press) section 2.2
+ * (16-token blocks, per-sequence block table mapping logical to physical
+ * blocks), section 2.3 (copy-on-write of a block whose reference count is
+ * above one), section 5.1 (exact attention combined by online softmax) and
+ * section 六 (decode loop: read the KV cache, attend, write the new token's
+ * K/V into its block); "vLLM：重塑大模型推理性能的关键引擎" (unionyoga.cn),
+ * PagedAttention section, kernel sketch (ceil(context_len / BLOCK_SIZE)
+ * blocks per sequence, table row stride MAX_BLOCKS).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every data pointer is a DEVICE pointer on the current CUDA device,
+ *   except the two pointer ARRAYS of pa_copy_blocks, which live in host
+ *   memory and hold device pointers.  The caller owns every buffer.
+ * - The library allocates nothing and never synchronises the stream: work
+ *   is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *   legacy default stream) and the call returns.
+ * - Element type of q, out, caches, key and value: 16-bit, fp16 or bf16
+ *   (pa_dims.dtype).  Arithmetic is fp32; outputs round to nearest-even.
+ * - Layouts (row-major, contiguous):
+ *     q, out         [num_seqs, num_heads, head_dim]
+ *     k/v cache      [num_blocks, num_kv_heads, block_size, head_dim]
+ *     block_tables   int32 [num_seqs, max_blocks_per_seq]
+ *     context_lens   int32 [num_seqs]
+ *     key, value     [num_tokens, num_kv_heads, head_dim]
+ *     slot_mapping   int64 [num_tokens]; slot = block * block_size + offset
+ *     block_mapping  int64 [num_pairs, 2]; (src block, dst block)
+ * - Query head h reads KV head h / (num_heads / num_kv_heads).
+ * - Supported: block_size 16, head_dim 64 or 128, num_heads / num_kv_heads
+ *   in {1, 2, 4, 8, 16}.  Data pointers must be 16-byte aligned.
+ * - Host-side argument errors return a negative pa_status before anything
+ *   is enqueued; pa_last_error() then describes the problem.
+ * - Device data (table entries, lengths, slots) is range-checked inside the
+ *   kernels: an out-of-range value is never dereferenced; it is replaced by
+ *   a safe value or skipped, and a bit is set in a device error word that
+ *   pa_device_error() returns.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_NULL = -1,        /* a required pointer is NULL */
+    PA_ERR_DTYPE = -2,       /* dtype is not PA_F16 / PA_BF16 */
+    PA_ERR_SHAPE = -3,       /* inconsistent or negative sizes */
+    PA_ERR_UNSUPPORTED = -4, /* block_size / head_dim / group size not built */
+    PA_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
+    PA_ERR_CUDA = -6,        /* a CUDA launch or query failed */
+    PA_ERR_ALIGN = -7        /* a data pointer is not 16-byte aligned */
+} pa_status;
+
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (pa_device_error). */
+#define PA_DEVERR_BLOCK_ID 1u    /* a block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT 2u     /* context_len < 0, above max_blocks_per_seq*16,
+                                    or above the max_context_len given */
+#define PA_DEVERR_SLOT 4u        /* a slot_mapping entry beyond the pool */
+#define PA_DEVERR_COPY_PAIR 8u   /* a block_mapping id outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 16u    /* a pipeline wait gave up (bounded spin) */
+
+typedef struct pa_dims {
+    int32_t num_seqs;           /* S: sequences in the batch */
+    int32_t num_heads;          /* H: query heads */
+    int32_t num_kv_heads;       /* Hk: KV heads (H % Hk == 0) */
+    int32_t head_dim;           /* D: 64 or 128 */
+    int32_t block_size;         /* B: tokens per block, 16 */
+    int32_t max_blocks_per_seq; /* MB: row stride of block_tables */
+    int64_t num_blocks;         /* NB: physical blocks in each cache */
+    int32_t dtype;              /* pa_dtype */
+} pa_dims;
+
+/*
+ * Bytes of device workspace pa_decode needs for these dims, the largest
+ * context length it will see and the partition size (0 = automatic; else a
+ * positive multiple of 16 tokens).  0 means no workspace is needed (every
+ * sequence fits in one partition).  Returns (size_t)-1 for invalid dims.
+ */
+size_t pa_decode_workspace_size(const pa_dims *dims, int32_t max_context_len,
+                                int32_t partition_tokens);
+
+/*
+ * Number of KV partitions per sequence pa_decode will use (1 = unsplit),
+ * or a negative pa_status for invalid arguments.
+ */
+int32_t pa_decode_num_partitions(const pa_dims *dims, int32_t max_context_len,
+                                 int32_t partition_tokens);
+
+/*
+ * Decode attention (ybb.press section 2.2 + 5.1; unionyoga.cn kernel sketch).
+ * For every sequence s and query head h, with n = context_lens[s] and
+ * K_s[j] = k_cache[block_tables[s, j / 16], h / (H / Hk), j % 16, :]:
+ *     out[s, h, :] = sum_{j < n} softmax_j(scale * q[s, h, :] . K_s[j]) V_s[j]
+ * A sequence with n == 0 gets an all-zero row.  Only the first
+ * ceil(n / 16) table entries and the first n slots are read.
+ *
+ * num_kv_heads must equal dims->num_kv_heads (it is the pages' explicit
+ * argument; the duplicate guards against a caller mixing layers).
+ * max_context_len is a host-known upper bound on context_lens (it sizes the
+ * partition grid); lengths above it are clamped and flagged.
+ * partition_tokens: 0 = automatic (512-token partitions once a context can
+ * exceed 512 tokens), else a positive multiple of 16; with more than one
+ * partition, partial results go to `workspace` (at least
+ * pa_decode_workspace_size() bytes, 256-byte aligned, contents ignored on
+ * entry) and a log-sum-exp merge kernel combines them.
+ * Enqueues one or two kernels on `stream`.
+ */
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, float scale,
+                    int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
+                    int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/*
+ * Cache write (ybb.press section 六, "write into the KV cache block").
+ * For every token t < num_tokens with slot = slot_mapping[t] >= 0 and every
+ * KV head h:
+ *     k_cache[slot / 16, h, slot % 16, :] = key[t, h, :]   (same for value)
+ * Negative slots are skipped (padding tokens).  Slots must be distinct: two
+ * tokens writing one slot race.  Bit-exact copy; one kernel on `stream`.
+ */
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                               const int64_t *slot_mapping, int32_t num_tokens,
+                               const pa_dims *dims, void *stream);
+
+/*
+ * Copy-on-write block duplication (ybb.press section 2.3).  For every layer
+ * l < num_layers and pair i < num_pairs, (src, dst) = block_mapping[i]:
+ *     k_caches[l][dst] = k_caches[l][src]   (all num_kv_heads * 16 * head_dim
+ *     v_caches[l][dst] = v_caches[l][src]    elements of the block)
+ * k_caches / v_caches are HOST arrays of num_layers device pointers, each
+ * cache shaped by dims.  block_mapping is a DEVICE array.  Pairs run
+ * concurrently: destinations must be distinct and no destination may also
+ * be a source.  Bit-exact; one kernel per 64 layers on `stream`.
+ */
+pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
+                         const int64_t *block_mapping, int32_t num_pairs, const pa_dims *dims,
+                         void *stream);
+
+/* Thread-local description of the last non-OK status returned on this
+ * thread ("" if none).  Owned by the library; valid until the next call. */
+const char *pa_last_error(void);
+
+/*
+ * Synchronises `stream`, then returns the device error word of the current
+ * device (a PA_DEVERR_* bit mask, 0 = clean) through *word and clears it.
+ * Returns PA_ERR_CUDA if the synchronisation or the read fails.
+ */
+pa_status pa_device_error(void *stream, uint32_t *word);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

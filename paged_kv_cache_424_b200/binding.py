@@ -1,0 +1,205 @@
+"""Python binding of ``libpa.so``: the C-ABI calls of ``include/pa.h`` with the
+same names, taking torch CUDA tensors.
+
+Argument marshalling only: shapes and dtypes are read off the tensors into a
+``pa_dims`` struct, pointers come from ``data_ptr()``, the stream from
+``torch.cuda.current_stream()`` unless one is given.  Every operation runs in
+the library's CUDA kernels; there is no fallback.  Importing this module
+loads the library and raises :class:`LibraryMissing` if it is not built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_OK = 0
+STATUS = {0: "PA_OK", -1: "PA_ERR_NULL", -2: "PA_ERR_DTYPE", -3: "PA_ERR_SHAPE", -4: "PA_ERR_UNSUPPORTED",
+          -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_CUDA", -7: "PA_ERR_ALIGN"}
+PA_F16, PA_BF16 = 0, 1
+DEVERR = {1: "BLOCK_ID", 2: "CONTEXT", 4: "SLOT", 8: "COPY_PAIR", 16: "TIMEOUT"}
+
+# The C entry points declared in include/pa.h, in declaration order.
+EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_reshape_and_cache",
+           "pa_copy_blocks", "pa_last_error", "pa_device_error", "pa_version"]
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class pa_dims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
+                ("num_blocks", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+def _load(path: str = LIB_PATH):
+    if not os.path.exists(path):
+        raise LibraryMissing(f"{path} is not built; run `python -m paged_kv_cache_424_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    dp = ctypes.POINTER(pa_dims)
+    lib.pa_decode_workspace_size.argtypes = [dp, i32, i32]
+    lib.pa_decode_workspace_size.restype = u64
+    lib.pa_decode_num_partitions.argtypes = [dp, i32, i32]
+    lib.pa_decode_num_partitions.restype = i32
+    lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, dp, i32, i32, vp, u64, vp]
+    lib.pa_decode.restype = ctypes.c_int
+    lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, dp, vp]
+    lib.pa_reshape_and_cache.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
+    lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_last_error.argtypes = []
+    lib.pa_last_error.restype = ctypes.c_char_p
+    lib.pa_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.pa_device_error.restype = ctypes.c_int
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    return lib
+
+
+LIB = _load()
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int) -> None:
+    if status != PA_OK:
+        raise PagedAttentionError(status, LIB.pa_last_error().decode(errors="replace"))
+
+
+def _need_cuda(*ts: Optional[torch.Tensor]) -> None:
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def make_dims(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+              max_blocks_per_seq: int, num_blocks: int, dtype: int) -> pa_dims:
+    return pa_dims(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype)
+
+
+def dims_of(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) -> pa_dims:
+    S, H, D = q.shape
+    NB, Hk, B, D2 = k_cache.shape
+    if D2 != D:
+        raise ValueError("q and k_cache disagree on head_dim")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    return make_dims(S, H, Hk, D, B, MB, NB, _dtype_code(q))
+
+
+def cache_dims(k_cache: torch.Tensor) -> pa_dims:
+    NB, Hk, B, D = k_cache.shape
+    return make_dims(0, Hk, Hk, D, B, 0, NB, _dtype_code(k_cache))
+
+
+# ---------------------------------------------------------------------------
+# the C-ABI calls
+# ---------------------------------------------------------------------------
+def pa_version() -> int:
+    return int(LIB.pa_version())
+
+
+def pa_last_error() -> str:
+    return LIB.pa_last_error().decode(errors="replace")
+
+
+def pa_decode_workspace_size(dims: pa_dims, max_context_len: int, partition_tokens: int = 0) -> int:
+    n = LIB.pa_decode_workspace_size(ctypes.byref(dims), int(max_context_len), int(partition_tokens))
+    if n == ctypes.c_size_t(-1).value:
+        raise PagedAttentionError(-3, pa_last_error())
+    return int(n)
+
+
+def pa_decode_num_partitions(dims: pa_dims, max_context_len: int, partition_tokens: int = 0) -> int:
+    n = int(LIB.pa_decode_num_partitions(ctypes.byref(dims), int(max_context_len), int(partition_tokens)))
+    if n < 0:
+        raise PagedAttentionError(n, pa_last_error())
+    return n
+
+
+def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
+              max_context_len: int, partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """out[s, h] = softmax(scale * q[s, h] . K_s^T) V_s over the paged cache."""
+    _need_cuda(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    dims = dims_of(q, k_cache, block_tables)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = LIB.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                       float(scale), int(num_kv_heads), ctypes.byref(dims), int(max_context_len),
+                       int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st)
+    return out
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                         slot_mapping: torch.Tensor, stream=None) -> None:
+    """k_cache[slot // 16, :, slot % 16] = key[t] (and V) for slot >= 0."""
+    _need_cuda(key, value, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    dims = cache_dims(k_cache)
+    st = LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                  int(slot_mapping.numel()), ctypes.byref(dims), _stream(stream))
+    _check(st)
+
+
+def pa_copy_blocks(k_caches: Sequence[torch.Tensor], v_caches: Sequence[torch.Tensor],
+                   block_mapping: torch.Tensor, stream=None) -> None:
+    """Per layer: block dst of K and V becomes a copy of block src."""
+    if len(k_caches) != len(v_caches) or not k_caches:
+        raise ValueError("need matching, non-empty lists of K and V caches")
+    _need_cuda(*k_caches, *v_caches, block_mapping)
+    if block_mapping.dtype != torch.int64:
+        raise TypeError("block_mapping must be int64")
+    L = len(k_caches)
+    kp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in k_caches])
+    vp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in v_caches])
+    dims = cache_dims(k_caches[0])
+    pairs = block_mapping.numel() // 2
+    st = LIB.pa_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), L,
+                            _ptr(block_mapping), int(pairs), ctypes.byref(dims), _stream(stream))
+    _check(st)
+
+
+def pa_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    w = ctypes.c_uint32(0)
+    _check(LIB.pa_device_error(_stream(stream), ctypes.byref(w)))
+    return int(w.value)

@@ -1,0 +1,212 @@
+// pa_api.cu -- the extern "C" entry points declared in include/pa.h: host-side
+// argument validation, the split-KV plan, and dispatch to the launchers.
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "../../include/pa.h"
+#include "pa_common.cuh"
+#include "pa_decode.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+pa_status fail(pa_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pa_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kAutoPartitionTokens = 512;
+constexpr int kMaxPartitionTokens = 32768;
+
+// Checks of the fields every call uses.  `attention` adds the query-side ones.
+pa_status check_dims(const pa_dims *d, bool attention) {
+    if (!d) return fail(PA_ERR_NULL, "dims is NULL");
+    if (d->dtype != PA_F16 && d->dtype != PA_BF16) return fail(PA_ERR_DTYPE, "dtype %d is not PA_F16/PA_BF16", d->dtype);
+    if (d->num_kv_heads <= 0 || d->head_dim <= 0 || d->block_size <= 0 || d->num_blocks <= 0)
+        return fail(PA_ERR_SHAPE, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
+    if (d->block_size != 16) return fail(PA_ERR_UNSUPPORTED, "block_size %d: only 16 is built", d->block_size);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are built", d->head_dim);
+    if (!attention) return PA_OK;
+    if (d->num_seqs < 0 || d->num_heads <= 0 || d->max_blocks_per_seq < 0)
+        return fail(PA_ERR_SHAPE, "num_seqs and max_blocks_per_seq must be >= 0, num_heads > 0");
+    if (d->num_seqs > 65535 || d->num_heads > 65535)
+        return fail(PA_ERR_SHAPE, "num_seqs and num_heads must be <= 65535 (grid limits)");
+    if (d->num_heads % d->num_kv_heads != 0)
+        return fail(PA_ERR_SHAPE, "num_heads %d is not a multiple of num_kv_heads %d", d->num_heads, d->num_kv_heads);
+    const int g = d->num_heads / d->num_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16)
+        return fail(PA_ERR_UNSUPPORTED, "group size %d: only 1, 2, 4, 8, 16 are built", g);
+    return PA_OK;
+}
+
+struct Plan {
+    int part_blocks = 1;
+    int max_parts = 1;
+    size_t o_bytes = 0;    // partial outputs
+    size_t lse_off = 0;    // offset of the lse array
+    size_t ws_bytes = 0;   // total workspace (0 when unsplit)
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl) {
+    if (max_context_len < 0) return fail(PA_ERR_SHAPE, "max_context_len %d < 0", max_context_len);
+    if ((int64_t)max_context_len > (int64_t)d->max_blocks_per_seq * d->block_size)
+        return fail(PA_ERR_SHAPE, "max_context_len %d exceeds max_blocks_per_seq * block_size = %lld", max_context_len,
+                    (long long)d->max_blocks_per_seq * d->block_size);
+    int P;
+    if (partition_tokens == 0) {
+        P = max_context_len > kAutoPartitionTokens ? kAutoPartitionTokens : max_context_len;
+    } else {
+        if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > kMaxPartitionTokens)
+            return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
+                        partition_tokens, kMaxPartitionTokens);
+        P = partition_tokens;
+    }
+    const int ctx_blocks = (max_context_len + 15) / 16;
+    int part_blocks = (P + 15) / 16;
+    if (part_blocks < 1) part_blocks = 1;
+    int max_parts = ctx_blocks == 0 ? 1 : (ctx_blocks + part_blocks - 1) / part_blocks;
+    if (max_parts == 1) part_blocks = ctx_blocks > 0 ? ctx_blocks : 1;  // one partition: size it to the context
+    pl->part_blocks = part_blocks;
+    pl->max_parts = max_parts;
+    if (max_parts > 1) {
+        const size_t rows = (size_t)d->num_seqs * d->num_heads * max_parts;
+        pl->o_bytes = align_up(rows * d->head_dim * sizeof(float), 256);
+        pl->lse_off = pl->o_bytes;
+        pl->ws_bytes = pl->o_bytes + align_up(rows * sizeof(float), 256);
+    }
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_last_error(void) { return g_err; }
+
+int32_t pa_version(void) { return 100; }
+
+size_t pa_decode_workspace_size(const pa_dims *dims, int32_t max_context_len, int32_t partition_tokens) {
+    if (check_dims(dims, true) != PA_OK) return (size_t)-1;
+    Plan pl;
+    if (make_plan(dims, max_context_len, partition_tokens, &pl) != PA_OK) return (size_t)-1;
+    return pl.ws_bytes;
+}
+
+int32_t pa_decode_num_partitions(const pa_dims *dims, int32_t max_context_len, int32_t partition_tokens) {
+    pa_status st = check_dims(dims, true);
+    if (st != PA_OK) return st;
+    Plan pl;
+    st = make_plan(dims, max_context_len, partition_tokens, &pl);
+    if (st != PA_OK) return st;
+    return pl.max_parts;
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    const int32_t *context_lens, float scale, int32_t num_kv_heads, const pa_dims *dims,
+                    int32_t max_context_len, int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                    void *stream) {
+    pa_status st = check_dims(dims, true);
+    if (st != PA_OK) return st;
+    if (num_kv_heads != dims->num_kv_heads)
+        return fail(PA_ERR_SHAPE, "num_kv_heads %d != dims->num_kv_heads %d", num_kv_heads, dims->num_kv_heads);
+    Plan pl;
+    st = make_plan(dims, max_context_len, partition_tokens, &pl);
+    if (st != PA_OK) return st;
+    if (dims->num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !context_lens || (!block_tables && dims->max_blocks_per_seq > 0))
+        return fail(PA_ERR_NULL, "a required pointer is NULL");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "out, q, k_cache and v_cache must be 16-byte aligned");
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes)
+            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.ws_bytes,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned16(workspace)) return fail(PA_ERR_ALIGN, "workspace must be 16-byte aligned");
+    }
+    pa::DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
+    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.lse_off) : nullptr;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.num_seqs = dims->num_seqs;
+    p.num_heads = dims->num_heads;
+    p.num_kv_heads = dims->num_kv_heads;
+    p.max_blocks_per_seq = dims->max_blocks_per_seq;
+    p.num_blocks = dims->num_blocks;
+    p.part_blocks = pl.part_blocks;
+    p.max_parts = pl.max_parts;
+    const int g = dims->num_heads / dims->num_kv_heads;
+    cudaError_t e = pa::launch_decode_simt(p, dims->dtype, dims->head_dim, g, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                               const int64_t *slot_mapping, int32_t num_tokens, const pa_dims *dims, void *stream) {
+    pa_status st = check_dims(dims, false);
+    if (st != PA_OK) return st;
+    if (num_tokens < 0) return fail(PA_ERR_SHAPE, "num_tokens %d < 0", num_tokens);
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return fail(PA_ERR_NULL, "a required pointer is NULL");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "key, value and caches must be 16-byte aligned");
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    cudaError_t e = pa::launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens, cd,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache launch");
+    return PA_OK;
+}
+
+pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
+                         const int64_t *block_mapping, int32_t num_pairs, const pa_dims *dims, void *stream) {
+    pa_status st = check_dims(dims, false);
+    if (st != PA_OK) return st;
+    if (num_layers < 0 || num_pairs < 0) return fail(PA_ERR_SHAPE, "num_layers and num_pairs must be >= 0");
+    if (num_layers == 0 || num_pairs == 0) return PA_OK;
+    if (!k_caches || !v_caches || !block_mapping) return fail(PA_ERR_NULL, "a required pointer is NULL");
+    for (int i = 0; i < num_layers; ++i) {
+        if (!k_caches[i] || !v_caches[i]) return fail(PA_ERR_NULL, "cache pointer of layer %d is NULL", i);
+        if (!aligned16(k_caches[i]) || !aligned16(v_caches[i]))
+            return fail(PA_ERR_ALIGN, "cache pointers of layer %d must be 16-byte aligned", i);
+    }
+    if (num_pairs > 65535) return fail(PA_ERR_SHAPE, "num_pairs %d > 65535", num_pairs);
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    cudaError_t e = pa::launch_copy_blocks(k_caches, v_caches, num_layers, block_mapping, num_pairs, cd,
+                                           static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_copy_blocks launch");
+    return PA_OK;
+}
+
+pa_status pa_device_error(void *stream, uint32_t *word) {
+    if (!word) return fail(PA_ERR_NULL, "word is NULL");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_device_error sync");
+    unsigned int w = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&w, pa::g_device_error, sizeof w);
+    if (e != cudaSuccess) return cuda_fail(e, "pa_device_error read");
+    e = cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "pa_device_error clear");
+    *word = w;
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,109 @@
+// pa_cache.cu -- the two companion kernels of paged decode:
+//
+// reshape_and_cache: "vLLM PagedAttention 大模型推理架构深度实战" section 六,
+//   decode loop step "write into the KV cache block": token t's key/value
+//   rows go to slot slot_mapping[t] = block * 16 + offset of the head-major
+//   pool [NB, Hk, 16, D].
+// copy_blocks: same page, section 2.3: a block shared by several sequences is
+//   copied before one of them writes into it (copy-on-write).
+//
+// Both are pure data movement (bit-exact) and HBM-bound: 16-byte vector
+// loads and stores, consecutive threads on consecutive 16-byte chunks.
+#include "pa_common.cuh"
+#include "pa_decode.h"
+
+namespace pa {
+
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kBlock = 16;
+constexpr int kCopyLayers = 64;  // layer pointers per copy_blocks launch
+
+// One thread per 16-byte chunk of a (token, kv head) row, for key and value.
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
+                             uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                             const int64_t *__restrict__ slot_mapping, int64_t num_items, int chunks_per_row,
+                             int num_kv_heads, int64_t num_slots) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= num_items) return;
+    const int64_t row = i / chunks_per_row;  // (token, kv head)
+    const int c = (int)(i % chunks_per_row);
+    const int64_t t = row / num_kv_heads;
+    const int h = (int)(row % num_kv_heads);
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;  // padding token
+    if (slot >= num_slots) {
+        if (h == 0 && c == 0) flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const int64_t blk = slot / kBlock, off = slot % kBlock;
+    const int64_t dst = ((blk * num_kv_heads + h) * kBlock + off) * chunks_per_row + c;
+    k_cache[dst] = key[i];
+    v_cache[dst] = value[i];
+}
+
+struct LayerPtrs {
+    uint4 *k[kCopyLayers];
+    uint4 *v[kCopyLayers];
+};
+
+// CTA = (pair, layer): copies the whole K block and V block.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(const LayerPtrs ptrs, const int64_t *__restrict__ block_mapping, int64_t chunks_per_block,
+                       int64_t num_blocks) {
+    const int pair = blockIdx.x, layer = blockIdx.y;
+    const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && layer == 0) flag_error(PA_DEVERR_COPY_PAIR);
+        return;
+    }
+    const uint4 *ks = ptrs.k[layer] + src * chunks_per_block;
+    const uint4 *vs = ptrs.v[layer] + src * chunks_per_block;
+    uint4 *kd = ptrs.k[layer] + dst * chunks_per_block;
+    uint4 *vd = ptrs.v[layer] + dst * chunks_per_block;
+    for (int64_t i = threadIdx.x; i < chunks_per_block; i += blockDim.x) {
+        const uint4 a = ks[i];
+        const uint4 b = vs[i];
+        kd[i] = a;
+        vd[i] = b;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,
+                                     cudaStream_t stream) {
+    const int chunks = d.head_dim / 8;
+    const int64_t items = (int64_t)num_tokens * d.num_kv_heads * chunks;
+    if (items == 0) return cudaSuccess;
+    const int64_t grid = (items + 255) / 256;
+    reshape_and_cache_kernel<<<(unsigned)grid, 256, 0, stream>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), static_cast<uint4 *>(k_cache),
+        static_cast<uint4 *>(v_cache), slot_mapping, items, chunks, d.num_kv_heads, d.num_blocks * kBlock);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
+                               const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
+                               cudaStream_t stream) {
+    if (num_pairs == 0 || num_layers == 0) return cudaSuccess;
+    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim / 8;
+    for (int l0 = 0; l0 < num_layers; l0 += kCopyLayers) {
+        const int nl = num_layers - l0 < kCopyLayers ? num_layers - l0 : kCopyLayers;
+        LayerPtrs ptrs = {};
+        for (int i = 0; i < nl; ++i) {
+            ptrs.k[i] = static_cast<uint4 *>(k_caches[l0 + i]);
+            ptrs.v[i] = static_cast<uint4 *>(v_caches[l0 + i]);
+        }
+        copy_blocks_kernel<<<dim3(num_pairs, nl), 256, 0, stream>>>(ptrs, block_mapping, chunks, d.num_blocks);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace pa

@@ -1,0 +1,48 @@
+// pa_decode.h -- private interface between the C ABI (pa_api.cu) and the
+// kernel launchers.  Not installed; the public interface is include/pa.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+constexpr int kMaxDevices = 64;
+
+// Everything a decode launch needs; passed by value as the kernel argument.
+struct DecodeParams {
+    void *out;                   // [S, H, D] fp16/bf16
+    const void *q;               // [S, H, D]
+    const void *k_cache;         // [NB, Hk, 16, D]
+    const void *v_cache;         // [NB, Hk, 16, D]
+    const int32_t *block_tables; // [S, MB]
+    const int32_t *context_lens; // [S]
+    float *ws_o;                 // [S, H, max_parts, D] partial outputs (split only)
+    float *ws_lse;               // [S, H, max_parts] log2-sum-exp per partial
+    float scale_log2;            // scale * log2(e)
+    int32_t num_seqs, num_heads, num_kv_heads, max_blocks_per_seq;
+    int64_t num_blocks;
+    int32_t part_blocks;         // table entries per KV partition
+    int32_t max_parts;           // partitions in the grid (gridDim.x)
+};
+
+// Dynamic shared memory of the CUDA-core kernel for these sizes.
+int decode_simt_smem_bytes(int head_dim, int group, int part_blocks);
+
+// CUDA-core decode (+ merge when max_parts > 1) on `stream`.
+cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, int head_dim, int group,
+                               cudaStream_t stream);
+
+// Cache kernels.
+struct CacheDims {
+    int32_t num_kv_heads, head_dim;
+    int64_t num_blocks;
+};
+cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,
+                                     cudaStream_t stream);
+cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
+                               const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
+                               cudaStream_t stream);
+
+}  // namespace pa

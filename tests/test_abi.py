@@ -1,0 +1,125 @@
+"""The C-ABI library: it builds, loads, exports every function include/pa.h
+declares, and rejects bad arguments on the host (no GPU needed: every call
+here returns before anything is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_424_b200 import build
+    build.build()
+    from paged_kv_cache_424_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(pa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("pa_decode", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_workspace_size",
+              "pa_last_error", "pa_device_error"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(so, n)]
+    assert not missing, f"declared but not exported: {missing}"
+    assert sorted(lib.EXPORTS) == declared_functions()
+
+
+def test_version(lib):
+    assert lib.pa_version() >= 100
+
+
+def _dims(lib, **kw):
+    base = dict(num_seqs=4, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16, max_blocks_per_seq=256,
+                num_blocks=1024, dtype=lib.PA_BF16)
+    base.update(kw)
+    return lib.pa_dims(**base)
+
+
+def test_workspace_plan(lib):
+    d = _dims(lib)
+    # short contexts fit one partition: no workspace
+    assert lib.pa_decode_num_partitions(d, 512, 0) == 1
+    assert lib.pa_decode_workspace_size(d, 512, 0) == 0
+    # automatic 512-token partitions above that
+    assert lib.pa_decode_num_partitions(d, 513, 0) == 2
+    assert lib.pa_decode_num_partitions(d, 4096, 0) == 8
+    ws = lib.pa_decode_workspace_size(d, 4096, 0)
+    rows = 4 * 32 * 8
+    assert ws >= rows * 128 * 4 + rows * 4
+    # explicit partition sizes
+    assert lib.pa_decode_num_partitions(d, 4096, 16) == 256
+    assert lib.pa_decode_num_partitions(d, 4096, 4096) == 1
+    assert lib.pa_decode_workspace_size(d, 4096, 4096) == 0
+    assert lib.pa_decode_num_partitions(d, 0, 0) == 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(block_size=32), -4), (dict(head_dim=96), -4), (dict(num_heads=24, num_kv_heads=8), -4),
+    (dict(num_heads=30), -3), (dict(dtype=7), -2), (dict(num_kv_heads=0), -3), (dict(num_seqs=-1), -3),
+    (dict(num_seqs=70000), -3),
+])
+def test_bad_dims_rejected(lib, kw, status):
+    d = _dims(lib, **kw)
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, 0) == status
+    assert lib.pa_last_error()
+
+
+def test_bad_partition_and_context(lib):
+    d = _dims(lib)
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, 24) == -3   # not a multiple of 16
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, -16) == -3
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, 65536) == -3
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 4097, 0) == -3   # > max_blocks_per_seq * 16
+    assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), -1, 0) == -3
+
+
+def _decode_raw(lib, d, ptrs, nkv=8, maxlen=1000, part=0, ws=None, wsb=0):
+    out, q, k, v, bt, cl = ptrs
+    return lib.LIB.pa_decode(out, q, k, v, bt, cl, ctypes.c_float(0.1), nkv, ctypes.byref(d), maxlen, part, ws,
+                             wsb, None)
+
+
+def test_decode_host_errors(lib):
+    d = _dims(lib)
+    good = [ctypes.c_void_p(0x10000)] * 6
+    assert _decode_raw(lib, d, [None] + good[1:]) == -1
+    assert _decode_raw(lib, d, good, nkv=4) == -3
+    assert _decode_raw(lib, d, good) == -5  # 1000 tokens -> 2 partitions, no workspace
+    assert "workspace" in lib.pa_last_error()
+    assert _decode_raw(lib, d, good, ws=ctypes.c_void_p(0x20000), wsb=16) == -5
+    bad = [ctypes.c_void_p(0x10008)] + good[1:]
+    assert _decode_raw(lib, d, bad, maxlen=100) == -7
+    d0 = _dims(lib, num_seqs=0)
+    assert _decode_raw(lib, d0, [None] * 6) == 0  # empty batch: nothing to do
+
+
+def test_cache_ops_host_errors(lib):
+    d = _dims(lib)
+    p = ctypes.c_void_p(0x10000)
+    L = lib.LIB
+    assert L.pa_reshape_and_cache(None, p, p, p, p, 4, ctypes.byref(d), None) == -1
+    assert L.pa_reshape_and_cache(p, p, p, p, p, -1, ctypes.byref(d), None) == -3
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, ctypes.byref(d), None) == 0
+    assert L.pa_reshape_and_cache(ctypes.c_void_p(0x10004), p, p, p, p, 4, ctypes.byref(d), None) == -7
+    arr = (ctypes.c_void_p * 2)(0x10000, None)
+    assert L.pa_copy_blocks(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p), 2, p, 3,
+                            ctypes.byref(d), None) == -1
+    assert L.pa_copy_blocks(None, None, 0, None, 0, ctypes.byref(d), None) == 0
+    assert L.pa_copy_blocks(None, None, 1, p, -1, ctypes.byref(d), None) == -3
+    assert L.pa_device_error(None, None) == -1

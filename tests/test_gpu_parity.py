@@ -1,0 +1,253 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every scenario runs its cache writes / copies (bit-exact against the oracle,
+and no byte outside the written blocks may change) and its decode step
+(within the tolerances in ``gpu_util``), at reduced sizes that span several
+partitions and ragged tails and at the full benchmark sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import MAX_ABS, compare, require_gpu, run_and_compare, widen
+from pins import Paged, narrow, rand_bits
+from pins import widen as widen_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+    from paged_kv_cache_424_b200 import build
+    build.build()
+    from paged_kv_cache_424_b200 import binding
+    assert binding.pa_device_error() == 0, "device error word set before the test"
+    yield
+    assert binding.pa_device_error() == 0, "a kernel flagged a device error"
+
+
+def W():
+    from paged_kv_cache_424_b200 import workload
+    return workload
+
+
+# ---------------------------------------------------------------------------
+# the five scenarios
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("P", [0, 16, 64])
+def test_tiny(P):
+    run_and_compare(W().tiny(0), partition_tokens=P)
+
+
+def test_tiny_against_brute_force():
+    from oracle import brute
+    from paged_kv_cache_424_b200.session import DeviceSession
+    from oracle.harness import OracleSession
+    sc = W().tiny(0)
+    st = sc.steps[0]
+    dev = DeviceSession(sc)
+    out = dev.run_step(st)
+    ses = OracleSession(sc)
+    ses.apply_cache_ops(st)
+    k, v = ses.pool.view()
+    rel = ses.pool.relabel_tables(st.block_tables, st.context_lens, 16)
+    ref = np.array(brute.paged_decode(st.q, k, v, rel, st.context_lens, sc.scale, "f16"))
+    compare(out, ref, "f16", "tiny vs brute force")
+
+
+@pytest.mark.parametrize("P", [0, 16, 512, 2048])
+def test_mha7b_reduced(P):
+    sc = W().mha7b(seed=11, num_seqs=8, min_len=1, max_len=1500, num_blocks=1024)
+    run_and_compare(sc, partition_tokens=P)
+
+
+def test_mha7b_full():
+    run_and_compare(W().mha7b())
+
+
+def test_gqa8b_reduced_three_steps():
+    sc = W().gqa8b(seed=12, num_seqs=32, num_steps=3, median=128, cap=1200, new_min=1, new_max=200,
+                   num_blocks=8192)
+    run_and_compare(sc)
+
+
+def test_gqa8b_full_two_steps():
+    run_and_compare(W().gqa8b(num_steps=2))
+
+
+def test_long70b_reduced():
+    sc = W().long70b(seed=13, num_seqs=2, context_len=4096 + 7, num_blocks=1024)
+    run_and_compare(sc)
+    run_and_compare(sc, partition_tokens=16)
+
+
+def test_long70b_full():
+    run_and_compare(W().long70b())
+
+
+@pytest.mark.parametrize("every", [False, True])
+def test_cow_full(every):
+    sc = W().cow(cow_every_sample=every)
+    npairs = sc.steps[0].block_mapping.shape[0]
+    assert npairs == (128 if every else 112)
+    dev, orc, _ = run_and_compare(sc)
+    # the shared prefix blocks are exactly as admitted (copy-on-write)
+    st = sc.steps[0]
+    pos = {int(b): i for i, b in enumerate(st.admit_ids)}
+    ids = torch.from_numpy(sc.shared_blocks).to(dev.k_cache.device)
+    got_k = dev.k_cache.view(torch.int16).index_select(0, ids).cpu().numpy().view(np.uint16)
+    want_k = st.admit_k[[pos[int(b)] for b in sc.shared_blocks]]
+    assert np.array_equal(got_k, want_k), "a shared prefix block was modified"
+
+
+@pytest.mark.parametrize("name", ["mha7b", "gqa8b"])
+def test_positive_values_variant(name):
+    """V ~ U[0, 1]: outputs are ~0.5, so a collapsed output cannot pass."""
+    if name == "mha7b":
+        sc = W().mha7b(seed=21, num_seqs=8, min_len=1, max_len=2048, num_blocks=1024, v_lo=0.0)
+    else:
+        sc = W().gqa8b(seed=22, num_seqs=16, median=512, cap=4096, num_blocks=4096, v_lo=0.0)
+    _, _, stats = run_and_compare(sc)
+    assert stats[0]["max_abs"] <= MAX_ABS[sc.dims.dtype]
+
+
+# ---------------------------------------------------------------------------
+# invariants and edge cases on the GPU path
+# ---------------------------------------------------------------------------
+def gpu_decode(p: Paged, scale: float, P: int = 0) -> torch.Tensor:
+    from paged_kv_cache_424_b200 import binding as pa
+    dt = torch.float16 if p.dtype == "f16" else torch.bfloat16
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(dt)  # noqa: E731
+    q, k, v = dev(p.q), dev(p.k_cache), dev(p.v_cache)
+    bt = torch.from_numpy(p.tables).cuda()
+    cl = torch.from_numpy(p.lens).cuda()
+    maxlen = int(p.lens.max()) if p.lens.size else 0
+    dims = pa.dims_of(q, k, bt)
+    nbytes = pa.pa_decode_workspace_size(dims, maxlen, P)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda") if nbytes else None
+    out = torch.full(q.shape, float("nan"), dtype=dt, device="cuda")
+    pa.pa_decode(out, q, k, v, bt, cl, scale, p.Hk, maxlen, P, ws)
+    torch.cuda.synchronize()
+    return out
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("g", [1, 2, 4, 8, 16])
+def test_group_sizes_and_head_dims(dtype, D, g, orc):
+    rng = np.random.default_rng(100 + g + D)
+    Hk = 2
+    lens = [1, 15, 16, 17, 250, 513, 1100]
+    p = Paged(rng, lens, Hk * g, Hk, D, dtype)
+    scale = float(np.float32(1 / np.sqrt(D)))
+    ref = p.run(orc, scale)
+    for P in (0, 16, 1104):
+        compare(gpu_decode(p, scale, P), ref, dtype, f"g={g} D={D} P={P}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_length_one_returns_v_bit_exact(dtype):
+    rng = np.random.default_rng(5)
+    p = Paged(rng, [1, 1, 1, 1], 8, 2, 128, dtype)
+    out = bits(gpu_decode(p, 0.1))
+    for s in range(4):
+        want = np.repeat(p.vs[s][0], 4, axis=0)  # [Hk, D] -> heads h // 4
+        assert np.array_equal(out[s], want), "length 1 must return V bit for bit"
+
+
+def test_zero_length_rows_are_zero():
+    rng = np.random.default_rng(6)
+    p = Paged(rng, [0, 37, 0, 600], 4, 4, 128, "bf16")
+    for P in (0, 16):
+        out = gpu_decode(p, 0.1, P)
+        assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
+        assert torch.isfinite(out[1]).all() and torch.isfinite(out[3]).all()
+
+
+def test_physical_permutation_invariance_bit_exact():
+    rng = np.random.default_rng(7)
+    p = Paged(rng, [300, 1000, 17], 32, 8, 128, "bf16")
+    a = bits(gpu_decode(p, 0.09))
+    NB = p.k_cache.shape[0]
+    perm = rng.permutation(NB)
+    k2, v2 = np.empty_like(p.k_cache), np.empty_like(p.v_cache)
+    k2[perm], v2[perm] = p.k_cache, p.v_cache
+    p.k_cache, p.v_cache = k2, v2
+    p.tables = perm[p.tables].astype(np.int32)
+    b = bits(gpu_decode(p, 0.09))
+    assert np.array_equal(a, b), "output depends on physical placement"
+
+
+def test_deterministic_across_runs():
+    rng = np.random.default_rng(8)
+    p = Paged(rng, [2000, 100, 700], 64, 8, 128, "bf16")
+    a = bits(gpu_decode(p, 0.09))
+    b = bits(gpu_decode(p, 0.09))
+    assert np.array_equal(a, b)
+
+
+def test_split_sizes_agree():
+    """Partitions of 16, 512 and the whole context give the same attention
+    (the log-sum-exp merge is exact up to fp32 rounding): within one output
+    ulp of each other."""
+    rng = np.random.default_rng(9)
+    p = Paged(rng, [4000, 33, 1500], 16, 2, 128, "f16")
+    outs = [widen(gpu_decode(p, 0.09, P)) for P in (16, 512, 4000 // 16 * 16 + 16)]
+    ulp = np.spacing(np.abs(outs[0]).astype(np.float16)).astype(np.float64)
+    for o in outs[1:]:
+        assert np.all(np.abs(o - outs[0]) <= ulp + 1e-7)
+
+
+def test_position_tagged_indirection():
+    """V encodes the logical position; one key dominates; the output must name
+    that position (proves the table lookup, slot and partition arithmetic)."""
+    rng = np.random.default_rng(10)
+    lens = [100, 17, 64, 33, 2000, 1025]
+    chosen = [0, 16, 63, 20, 1999, 512]
+    D, H, Hk = 128, 8, 2
+    q = rand_bits(rng, (len(lens), H, D), "f16", -0.5, 0.5)
+    ks, vs = [], []
+    for s, L in enumerate(lens):
+        k = rand_bits(rng, (L, Hk, D), "f16", -0.1, 0.1)
+        for h in range(Hk):
+            k[chosen[s], h] = narrow(8.0 * widen_bits(q[s, h * (H // Hk)], "f16"), "f16")
+        v = np.zeros((L, Hk, D))
+        v[:, :, 0] = (np.arange(L) / 2048.0)[:, None]
+        ks.append(k)
+        vs.append(narrow(v, "f16"))
+    p = Paged(rng, lens, H, Hk, D, "f16", q=q, ks=ks, vs=vs)
+    for P in (0, 16):
+        out = widen(gpu_decode(p, 1.0, P))
+        for s in range(len(lens)):
+            for h in range(0, H, H // Hk):
+                assert round(out[s, h, 0] * 2048) == chosen[s], (s, h, out[s, h, 0] * 2048)
+
+
+def test_device_error_word_reports_bad_inputs():
+    """Out-of-range table entries, lengths and slots are caught by the kernels'
+    own range checks (never dereferenced) and reported in the error word."""
+    from paged_kv_cache_424_b200 import binding as pa
+    rng = np.random.default_rng(11)
+    p = Paged(rng, [40, 20], 4, 4, 128, "bf16")
+    p.tables[0, 1] = 10 ** 6
+    gpu_decode(p, 0.1)
+    assert pa.pa_device_error() & 1
+    p.tables[0, 1] = 0
+    p.lens = np.array([40, 20], np.int32)
+    dt = torch.bfloat16
+    k = torch.zeros((4, 4, 16, 128), dtype=dt, device="cuda")
+    v = torch.zeros_like(k)
+    key = torch.ones((2, 4, 128), dtype=dt, device="cuda")
+    slots = torch.tensor([5, 4 * 16], dtype=torch.int64, device="cuda")  # second one is past the pool
+    pa.pa_reshape_and_cache(key, key, k, v, slots)
+    assert pa.pa_device_error() & 4
+    assert k[0, :, 5].eq(1).all() and k[1:].eq(0).all() and k[0, :, :5].eq(0).all()
+    bm = torch.tensor([[0, 2], [1, 99]], dtype=torch.int64, device="cuda")
+    pa.pa_copy_blocks([k], [v], bm)
+    assert pa.pa_device_error() & 8
+    assert torch.equal(k[2], k[0])
