@@ -130,6 +130,39 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     void *stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  The paper has no counterpart: this is a library convenience.
+ *
+ * Some callers have no way to hand pa_decode a workspace: a serving engine
+ * that has already given nearly all of HBM to its KV-cache pool and forbids
+ * further allocations, a plugin running inside a host framework whose memory
+ * pool it may not touch, or code on a path where cudaMalloc's implicit
+ * device synchronisation is not acceptable.  This entry point takes the same
+ * arguments as pa_decode minus the workspace and uses instead a scratch
+ * array that the library itself holds in device memory: 64 MiB
+ * (67108864 bytes), reserved on every GPU that loads the library until the
+ * process exits.
+ *
+ * - A call whose split-KV plan needs more than 64 MiB (see
+ *   pa_decode_workspace_size) returns PA_ERR_WORKSPACE with a message and
+ *   enqueues nothing; use pa_decode, larger partitions or fewer sequences.
+ * - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ * - The first call on each device that needs scratch looks up the array's
+ *   device address (cudaGetSymbolAddress, with that device current) and
+ *   keeps it; make that first call before any stream capture.
+ * - All calls on a device share the one array, which keeps the last call's
+ *   contents.  Nothing in it needs to start at zero (each call writes every
+ *   partial result it later reads), but calls whose kernels overlap on the
+ *   GPU (different streams, or several host threads) race on it: order them
+ *   on one stream or use pa_decode with separate workspaces.
+ * Results are those of pa_decode with the same arguments.
+ */
+pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, const int32_t *context_lens, float scale,
+                            int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
+                            int32_t partition_tokens, void *stream);
+
+/*
  * Cache write (ybb.press section 六, "write into the KV cache block").
  * For every token t < num_tokens with slot = slot_mapping[t] >= 0 and every
  * KV head h:

@@ -25,7 +25,8 @@ PA_F16, PA_BF16 = 0, 1
 DEVERR = {1: "BLOCK_ID", 2: "CONTEXT", 4: "SLOT", 8: "COPY_PAIR", 16: "TIMEOUT"}
 
 # The C entry points declared in include/pa.h, in declaration order.
-EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_reshape_and_cache",
+EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_decode_noalloc",
+           "pa_reshape_and_cache",
            "pa_copy_blocks", "pa_last_error", "pa_device_error", "pa_version"]
 
 
@@ -57,6 +58,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_num_partitions.restype = i32
     lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, dp, i32, i32, vp, u64, vp]
     lib.pa_decode.restype = ctypes.c_int
+    lib.pa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, dp, i32, i32, vp]
+    lib.pa_decode_noalloc.restype = ctypes.c_int
     lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, dp, vp]
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
@@ -164,6 +167,23 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
     st = LIB.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
                        float(scale), int(num_kv_heads), ctypes.byref(dims), int(max_context_len),
                        int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st)
+    return out
+
+
+def pa_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
+                      max_context_len: int, partition_tokens: int = 0, stream=None) -> torch.Tensor:
+    """pa_decode without a workspace argument: the split-KV scratch is the
+    library's own 64 MiB device array, for callers that cannot allocate.
+    Calls that overlap on the GPU race on that shared scratch."""
+    _need_cuda(out, q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    dims = dims_of(q, k_cache, block_tables)
+    st = LIB.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                               _ptr(context_lens), float(scale), int(num_kv_heads), ctypes.byref(dims),
+                               int(max_context_len), int(partition_tokens), _stream(stream))
     _check(st)
     return out
 

@@ -93,6 +93,11 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
 
 }  // namespace
 
+namespace pa {
+// Lets other entry points of the library report through pa_last_error().
+pa_status set_last_error(pa_status st, const char *msg) { return fail(st, "%s", msg); }
+}  // namespace pa
+
 extern "C" {
 
 const char *pa_last_error(void) { return g_err; }

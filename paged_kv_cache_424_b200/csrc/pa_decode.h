@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/pa.h"
+
 namespace pa {
 
 constexpr int kMaxDevices = 64;
@@ -25,6 +27,9 @@ struct DecodeParams {
     int32_t part_blocks;         // table entries per KV partition
     int32_t max_parts;           // partitions in the grid (gridDim.x)
 };
+
+// Record `msg` as the text pa_last_error() returns on this thread; returns st.
+pa_status set_last_error(pa_status st, const char *msg);
 
 // Dynamic shared memory of the CUDA-core kernel for these sizes.
 int decode_simt_smem_bytes(int head_dim, int group, int part_blocks);
