@@ -28,15 +28,29 @@ struct DecodeParams {
     int32_t max_parts;           // partitions in the grid (gridDim.x)
 };
 
+// Raise a kernel's dynamic shared-memory limit on the current device when a
+// launch needs more than was set before (the attribute is per device).
+template <typename K>
+inline cudaError_t ensure_smem(K kern, int bytes, int *configured_per_device) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (bytes > 48 * 1024 && bytes > configured_per_device[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        configured_per_device[dev] = bytes;
+    }
+    return cudaSuccess;
+}
+
 // Record `msg` as the text pa_last_error() returns on this thread; returns st.
 pa_status set_last_error(pa_status st, const char *msg);
 
-// Dynamic shared memory of the CUDA-core kernel for these sizes.
-int decode_simt_smem_bytes(int head_dim, int group, int part_blocks);
+// Fixed-partition decode (+ merge when max_parts > 1) on `stream`.
+cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group,
+                                      cudaStream_t stream);
 
-// CUDA-core decode (+ merge when max_parts > 1) on `stream`.
-cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, int head_dim, int group,
-                               cudaStream_t stream);
 
 // Cache kernels.
 struct CacheDims {
