@@ -76,6 +76,7 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_SLOT 4u        /* a slot_mapping entry beyond the pool */
 #define PA_DEVERR_COPY_PAIR 8u   /* a block_mapping id outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 16u    /* a pipeline wait gave up (bounded spin) */
+#define PA_DEVERR_LAYOUT 32u     /* internal shared-memory alignment check failed */
 
 typedef struct pa_dims {
     int32_t num_seqs;           /* S: sequences in the batch */

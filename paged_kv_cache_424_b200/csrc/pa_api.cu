@@ -157,8 +157,10 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
     p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.lse_off) : nullptr;
     const int g = dims->num_heads / dims->num_kv_heads;
-    cudaError_t e =
-        pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, g, static_cast<cudaStream_t>(stream));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = pa::decode_tc_supported(dims->head_dim, g, dims->num_blocks, dims->num_kv_heads)
+                        ? pa::launch_decode_tc(p, dims->dtype, g, cs)
+                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, g, cs);
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     return PA_OK;
 }

@@ -29,6 +29,7 @@ template <> struct Elem<__half> {
         return __half22float2(h);
     }
     static __device__ __forceinline__ __half from_float(float x) { return __float2half_rn(x); }
+    static __device__ __forceinline__ float to_float(__half x) { return __half2float(x); }
 };
 template <> struct Elem<__nv_bfloat16> {
     using T2 = __nv_bfloat162;
@@ -40,6 +41,7 @@ template <> struct Elem<__nv_bfloat16> {
         return r;
     }
     static __device__ __forceinline__ __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+    static __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 };
 
 // ---------------------------------------------------------------------------

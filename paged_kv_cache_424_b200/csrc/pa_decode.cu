@@ -20,6 +20,8 @@
 //   output; otherwise it writes (o_p, log2-sum-exp_p) to the workspace and
 //   the merge kernel combines partitions:
 //     out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M),  M = max_p lse_p.
+#include <type_traits>
+
 #include "pa_common.cuh"
 #include "pa_decode.h"
 #include "pa_simt.cuh"
@@ -210,8 +212,7 @@ cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
     kern<<<grid, kWarps * 32, smem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.max_parts == 1) return e;
-    merge_part_kernel<T, D><<<dim3(p.num_heads, p.num_seqs), D, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, D, stream);
 }
 
 template <typename T, int D>
@@ -227,6 +228,18 @@ cudaError_t launch_part_d(const DecodeParams &p, int group, cudaStream_t stream)
 }
 
 }  // namespace
+
+cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream) {
+    const dim3 grid(p.num_heads, p.num_seqs);
+    if (dtype == PA_F16) {
+        if (head_dim == 64) merge_part_kernel<__half, 64><<<grid, 64, 0, stream>>>(p);
+        else merge_part_kernel<__half, 128><<<grid, 128, 0, stream>>>(p);
+    } else {
+        if (head_dim == 64) merge_part_kernel<__nv_bfloat16, 64><<<grid, 64, 0, stream>>>(p);
+        else merge_part_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group,
                                       cudaStream_t stream) {

@@ -52,6 +52,14 @@ cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head
                                       cudaStream_t stream);
 
 
+// Log-sum-exp merge of the partitions written to the workspace.
+cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream);
+
+// Tensor-core decode for GQA groups (head_dim 128, group 4, 8 or 16) and
+// whether it applies to these sizes.
+bool decode_tc_supported(int head_dim, int group, int64_t num_blocks, int num_kv_heads);
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int group, cudaStream_t stream);
+
 // Cache kernels.
 struct CacheDims {
     int32_t num_kv_heads, head_dim;

@@ -1,0 +1,426 @@
+// pa_decode_tc.cu -- paged decode attention for GQA groups (4, 8 or 16 query
+// heads per KV head, head_dim 128) on the 5th-generation tensor cores.
+//
+// Method: "vLLM PagedAttention 大模型推理架构深度实战" section 2.2 (16-token
+// blocks reached through the block table) and section 5.1 (exact attention,
+// tiles combined by online softmax).  With a query group of G heads sharing
+// one KV head, a chunk of 128 cached tokens gives two real dense products:
+//   S (128 tokens x 16)  = K (128 x 128 dims) . Q^T (128 x 16)     [QK^T]
+//   O^T (128 dims x 16)  = V^T (128 x 128 tokens) . P^T (128 x 16)  [PV]
+// (the G query rows padded to the MMA's N = 16).
+//
+// CTA = (512-token partition, KV head, sequence): 6 warps.
+//   warp 4  producer: per chunk, 2-D tiled TMA loads of the 8 blocks' K rows
+//           and V rows (16 rows x 64 dims per box, 128-byte swizzle) into the
+//           K tile and the V tile; blocks past the partition are loaded from
+//           an out-of-range row, which the TMA fills with zeros.
+//   warp 5  MMA issuer (one thread): S into TMEM (double-buffered), then
+//           O = V^T P^T into TMEM (double-buffered), each completion signalled
+//           by tcgen05.commit on an mbarrier; allocates / frees TMEM.
+//   warps 0-3 softmax: thread t owns TMEM lane t = token t of S and output
+//           dim t of O.  Masks tokens past the context, keeps the online
+//           softmax with a lazy running max (raised only when a chunk's max
+//           beats it by 2^8), writes P (same 16-bit type as V) into a swizzled
+//           tile, and accumulates O chunk by chunk in registers.
+// Shared memory: K tile 32 KiB + V tile 32 KiB + Q 4 KiB + P 4 KiB (+ <1 KiB)
+// = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
+// Results go to `out` (one partition) or to the split workspace for the
+// log-sum-exp merge, exactly like the CUDA-core kernel.
+#include <mutex>
+#include <type_traits>
+
+#include "pa_common.cuh"
+#include "pa_decode.h"
+#include "pa_simt.cuh"
+#include "pa_tc.cuh"
+
+namespace pa {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kN = 16;              // MMA N: query heads padded to 16
+constexpr int kChunk = 128;         // tokens per chunk (MMA M)
+constexpr int kChunkBlocks = kChunk / kBlock;
+constexpr int kThreadsTc = 192;
+constexpr int kRegion = kChunk * 128;   // one 64-dim half of a K or V tile (bytes)
+
+// Shared-memory layout (bytes from the 1024-aligned base).
+constexpr int kKOff = 0;
+constexpr int kVOff = kKOff + 2 * kRegion;      // 32768
+constexpr int kQOff = kVOff + 2 * kRegion;      // 65536
+constexpr int kPOff = kQOff + 2 * kN * 128;     // 69632
+constexpr int kRedOff = kPOff + 2 * kN * 128;   // 73728: [2][4][16] floats
+constexpr int kBarOff = kRedOff + 2 * 4 * kN * 4;
+constexpr int kNumBars = 9;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;
+constexpr int kSmemTc = kMiscOff + 16;
+
+// TMEM columns: S buffers at 0 and 16, O buffers at 32 and 48.
+constexpr uint32_t kTmemCols = 64;
+__device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * kN); }
+__device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)(2 * kN + b * kN); }
+
+__device__ __forceinline__ int part_lmax_tc(const DecodeParams &p) {
+    return min(p.max_blocks_per_seq * kBlock, p.max_parts * p.part_blocks * kBlock);
+}
+
+__device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
+
+// Bounded wait that gives up at once when another thread already failed.
+__device__ __forceinline__ bool wait_ok(uint64_t *bar, uint32_t parity, int *fail) {
+    if (is_failed(fail)) return false;
+    if (mbar_wait(bar, parity)) return true;
+    atomicOr(fail, 1);
+    return false;
+}
+
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kThreadsTc, 3)
+    decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
+    using E = Elem<T>;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char *k_t = smem + kKOff;
+    unsigned char *v_t = smem + kVOff;
+    unsigned char *q_t = smem + kQOff;
+    unsigned char *p_t = smem + kPOff;
+    float *red = reinterpret_cast<float *>(smem + kRedOff);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    uint64_t *k_full = bars + 0, *k_empty = bars + 1, *v_full = bars + 2, *v_empty = bars + 3;
+    uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMiscOff);
+    int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
+
+    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.num_heads, head0 = kvh * G;
+    T *out = reinterpret_cast<T *>(p.out);
+
+    const int L = checked_len(p, s, part_lmax_tc(p), part == 0 && kvh == 0 && tid == 0);
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
+    if (part >= nparts) return;
+    const bool direct = nparts == 1;
+    if (L == 0) {
+        for (int i = tid; i < G * kD; i += blockDim.x)
+            out[((int64_t)s * H + head0 + i / kD) * kD + i % kD] = E::from_float(0.f);
+        return;
+    }
+    // The swizzled tiles need a 1024-byte aligned base; never touch them otherwise.
+    if (smem_addr(smem) & 1023u) {
+        if (tid == 0) flag_error(PA_DEVERR_LAYOUT);
+        return;
+    }
+    const int b0 = part * p.part_blocks;
+    const int nb = min(p.part_blocks, nblk - b0);          // blocks of this partition
+    const int nch = (nb + kChunkBlocks - 1) / kChunkBlocks; // chunks of 128 tokens
+    const int tok0 = b0 * kBlock;
+    const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
+
+    // ---- set-up -----------------------------------------------------------------
+    if (warp == 5) tc::tmem_alloc(tmem_slot, kTmemCols);
+    if (tid == 0) {
+        *fail = 0;
+        mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(&o_full[0], 1);
+        mbar_init(&o_full[1], 1);
+        mbar_init(p_full, 128);
+        fence_mbar_init();
+    }
+    if (tid < 128) {
+        // Q tile: rows = the group's query heads (zero rows up to 16), K-major
+        // 128-byte swizzle, two 64-dim regions.
+        const T *q = reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * kD;
+        for (int i = tid; i < kN * (kD / 8); i += 128) {
+            const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r < G) v = *reinterpret_cast<const uint4 *>(q + r * kD + c16 * 8);
+            *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
+        }
+        fence_proxy_async_smem();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------ producer ------------------------------
+        const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
+        for (int c = 0; c < nch; ++c) {
+            const int bi = c * kChunkBlocks + lane;
+            int y = oob_row;
+            if (lane < kChunkBlocks && bi < nb) y = (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock);
+            bool ok = true;
+            if (lane == 0) {
+                ok = c == 0 || wait_ok(k_empty, (c - 1) & 1, fail);
+                if (ok) mbar_arrive_expect_tx(k_full, 2 * kRegion);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < kChunkBlocks) {
+                tc::tma_load_2d(k_t + lane * 2048, &tmap_k, 0, y, k_full);
+                tc::tma_load_2d(k_t + kRegion + lane * 2048, &tmap_k, 64, y, k_full);
+            }
+            if (lane == 0) {
+                ok = c == 0 || wait_ok(v_empty, (c - 1) & 1, fail);
+                if (ok) mbar_arrive_expect_tx(v_full, 2 * kRegion);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane < kChunkBlocks) {
+                tc::tma_load_2d(v_t + lane * 2048, &tmap_v, 0, y, v_full);
+                tc::tma_load_2d(v_t + kRegion + lane * 2048, &tmap_v, 64, y, v_full);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = tc::instr_desc_f16(kBf16, false, kChunk, kN);
+            constexpr uint32_t idesc_pv = tc::instr_desc_f16(kBf16, true, kD, kN);
+            const uint32_t kb = smem_addr(k_t), vb = smem_addr(v_t), qb = smem_addr(q_t), pb = smem_addr(p_t);
+            auto pv = [&](int c) -> bool {
+                if (!wait_ok(p_full, c & 1, fail) || !wait_ok(v_full, c & 1, fail)) return false;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kChunk / 16; ++kk) {
+                    const uint64_t a = tc::smem_desc(vb + kk * 2048, kRegion, 1024);
+                    const uint64_t b = tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+                    tc::mma_f16(tmem + o_col(c & 1), a, b, idesc_pv, kk > 0);
+                }
+                tc::commit(&o_full[c & 1]);
+                tc::commit(v_empty);
+                return true;
+            };
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                ok = wait_ok(k_full, c & 1, fail);
+                if (!ok) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = tc::smem_desc(kb + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
+                    const uint64_t b = tc::smem_desc(qb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+                    tc::mma_f16(tmem + s_col(c & 1), a, b, idesc_qk, kk > 0);
+                }
+                tc::commit(&s_full[c & 1]);
+                tc::commit(k_empty);
+                if (c >= 1) ok = pv(c - 1);
+            }
+            if (ok) pv(nch - 1);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------ softmax warps ------------------------------
+        const int t = tid;                                      // token of S, dim of O
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // TMEM lane quadrant
+        float m[G], l[G], acc[G], alpha_prev[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+            acc[h] = 0.f;
+            alpha_prev[h] = 1.f;
+        }
+        auto epilogue = [&](int c) {
+            if (!wait_ok(&o_full[c & 1], (c >> 1) & 1, fail)) return;
+            tc::fence_after_sync();
+            float o[16];
+            tc::tmem_ld16(tmem + lane_base + o_col(c & 1), o);
+#pragma unroll
+            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha_prev[h], o[h]);
+        };
+        const bool has_tail = (b0 + nb == nblk) && (L % kBlock) != 0;  // partial last block here
+        for (int c = 0; c < nch; ++c) {
+            float x[G];
+            const int tok = tok0 + c * kChunk + t;
+            const bool valid = tok < tok_end;
+            bool ok = wait_ok(&s_full[c & 1], (c >> 1) & 1, fail);
+            if (ok) {
+                tc::fence_after_sync();
+                float sv[16];
+                tc::tmem_ld16(tmem + lane_base + s_col(c & 1), sv);
+#pragma unroll
+                for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+            } else {
+#pragma unroll
+                for (int h = 0; h < G; ++h) x[h] = -INFINITY;
+            }
+            // chunk max per head: warp max, then across the 4 warps
+            float *rc = red + (c & 1) * 4 * kN;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float v = x[h];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (lane == 0) rc[warp * kN + h] = v;
+            }
+            softmax_sync();
+            float alpha[G];
+            T pv[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float cm = fmaxf(fmaxf(rc[h], rc[kN + h]), fmaxf(rc[2 * kN + h], rc[3 * kN + h]));
+                alpha[h] = 1.f;
+                if (cm > m[h] + kLazyMax) {  // uniform across the 128 threads
+                    alpha[h] = ex2(m[h] - cm);
+                    l[h] *= alpha[h];
+                    m[h] = cm;
+                }
+                pv[h] = E::from_float(ex2(x[h] - m[h]));
+                l[h] += E::to_float(pv[h]);  // the rounded weight the MMA sees
+            }
+            if (c > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
+#pragma unroll
+            for (int h = 0; h < G; ++h) alpha_prev[h] = alpha[h];
+            if (c == nch - 1 && has_tail && ok) {
+                // Rows of the partial last block past the context come from the
+                // pool and may hold anything (NaN): zero them in the V tile
+                // once it has landed, so 0 * V stays 0 in the PV product.
+                if (wait_ok(v_full, c & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<uint4 *>(v_t + j * kRegion + t * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            // P tile: K-major, rows = heads, columns = tokens (two 64-token regions)
+            unsigned char *pr = p_t + (t >> 6) * (kN * 128);
+#pragma unroll
+            for (int h = 0; h < kN; ++h) {
+                const T v = h < G ? pv[h < G ? h : 0] : E::from_float(0.f);
+                *reinterpret_cast<T *>(pr + tc::sw128_offset(h, t & 63)) = v;
+            }
+            fence_proxy_async_smem();
+            tc::fence_before_sync();
+            mbar_arrive(p_full);
+        }
+        epilogue(nch - 1);
+
+        // l: per-thread partial sums over this thread's tokens -> total per head
+        float *rl = red;  // both halves of the chunk-max buffer are free now
+        softmax_sync();
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float v = l[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) rl[warp * kN + h] = v;
+        }
+        softmax_sync();
+        if (!is_failed(fail)) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float lt = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
+                const float o = acc[h] / lt;
+                if (direct) {
+                    out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
+                } else {
+                    const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
+                    p.ws_o[r * kD + t] = o;
+                    if (t == 0) p.ws_lse[r] = m[h] + log2f(lt);
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 5) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// A cache [NB, Hk, 16, 128] seen as rows of 128 elements; boxes of 16 rows
+// x 64 elements with the 128-byte swizzle; out-of-range rows read as zero.
+bool encode_cache_map(CUtensorMap *map, const void *base, int64_t rows, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int G>
+cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
+    const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
+    CUtensorMap tk, tv;
+    if (!encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) ||
+        !encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value))
+        return cudaErrorInvalidValue;
+    auto kern = decode_tc_kernel<T, G>;
+    static int configured[kMaxDevices] = {};
+    static int carveout_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices && !carveout_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        carveout_set[dev] = 1;
+    }
+    e = ensure_smem(kern, kSmemTc, configured);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.max_parts, p.num_kv_heads, p.num_seqs);
+    kern<<<grid, kThreadsTc, kSmemTc, stream>>>(p, tk, tv, (int)rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.max_parts == 1) return e;
+    return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
+}
+
+template <typename T>
+cudaError_t launch_tc_d(const DecodeParams &p, int group, cudaStream_t stream) {
+    switch (group) {
+        case 4: return launch_tc_t<T, 4>(p, stream);
+        case 8: return launch_tc_t<T, 8>(p, stream);
+        case 16: return launch_tc_t<T, 16>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool decode_tc_supported(int head_dim, int group, int64_t num_blocks, int num_kv_heads) {
+    return head_dim == kD && (group == 4 || group == 8 || group == 16) &&
+           num_blocks * num_kv_heads * kBlock < ((int64_t)1 << 31) - kBlock;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int group, cudaStream_t stream) {
+    return dtype == PA_F16 ? launch_tc_d<__half>(p, group, stream) : launch_tc_d<__nv_bfloat16>(p, group, stream);
+}
+
+}  // namespace pa

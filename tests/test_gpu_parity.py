@@ -198,16 +198,23 @@ def test_deterministic_across_runs():
     assert np.array_equal(a, b)
 
 
-def test_split_sizes_agree():
-    """Partitions of 16, 512 and the whole context give the same attention
-    (the log-sum-exp merge is exact up to fp32 rounding): within one output
-    ulp of each other."""
+@pytest.mark.parametrize("H,Hk,atol", [(4, 2, 0.0), (16, 2, 5e-4)])
+def test_split_sizes_agree(H, Hk, atol):
+    """Partitions of 16, 512 and the whole context give the same attention:
+    the log-sum-exp merge is exact up to fp32 rounding, so on the CUDA-core
+    path (group 2) the results agree within one output ulp.  On the
+    tensor-core path (group 8) P enters the PV product rounded to 16 bits
+    relative to a running max that depends on the split, which moves the
+    output by ~2^-11 |v| / sqrt(n): ~1e-5 at 4000 tokens, ~1e-4 at 33.  A
+    wrong merge would be off by ~1e-2; allow `atol` (a quarter of the fp16
+    parity tolerance) on that path."""
     rng = np.random.default_rng(9)
-    p = Paged(rng, [4000, 33, 1500], 16, 2, 128, "f16")
+    p = Paged(rng, [4000, 33, 1500], H, Hk, 128, "f16")
     outs = [widen(gpu_decode(p, 0.09, P)) for P in (16, 512, 4000 // 16 * 16 + 16)]
     ulp = np.spacing(np.abs(outs[0]).astype(np.float16)).astype(np.float64)
     for o in outs[1:]:
-        assert np.all(np.abs(o - outs[0]) <= ulp + 1e-7)
+        excess = np.abs(o - outs[0]) - ulp - atol
+        assert np.all(excess <= 1e-7), f"max difference beyond the bound: {excess.max():.3e}"
 
 
 def test_position_tagged_indirection():
