@@ -122,7 +122,10 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
     const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
 
     // ---- set-up -----------------------------------------------------------------
-    if (warp == 5) tc::tmem_alloc(tmem_slot, kTmemCols);
+    if (warp == 5) {
+        tc::tmem_alloc(tmem_slot, kTmemCols);
+        tc::tmem_relinquish();
+    }
     if (tid == 0) {
         *fail = 0;
         mbar_init(k_full, 1);
