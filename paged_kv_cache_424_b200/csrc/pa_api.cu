@@ -26,10 +26,13 @@ pa_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Automatic partition size: 512 tokens (32 blocks).  Long contexts then give
-// thousands of equal work items (an even load across the 148 SMs at 3 CTAs
-// per SM) for a merge that costs ~1% of the KV traffic.
-constexpr int kAutoPartitionTokens = 512;
+// Automatic partition size, measured on B200: 512 tokens for the CUDA-core
+// kernel (its per-warp rings favour many short items), 1024 tokens (8 chunks
+// of 128) for the tensor-core kernel, whose per-CTA set-up (TMEM, barriers,
+// Q tile) then amortises over more chunks while long contexts still give
+// thousands of CTAs.  The merge costs ~1-2% of the KV traffic either way.
+constexpr int kAutoPartitionSimt = 512;
+constexpr int kAutoPartitionTc = 1024;
 constexpr int kMaxPartitionTokens = 32768;
 
 // Checks of the fields every call uses.  `attention` adds the query-side ones.
@@ -72,7 +75,9 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
     if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > kMaxPartitionTokens)
         return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
                     partition_tokens, kMaxPartitionTokens);
-    const int P = partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
+    const int g = d->num_heads / d->num_kv_heads;
+    const bool tc = pa::decode_tc_supported(d->head_dim, g, d->num_blocks, d->num_kv_heads);
+    const int P = partition_tokens != 0 ? partition_tokens : tc ? kAutoPartitionTc : kAutoPartitionSimt;
     const int ctx_blocks = (max_context_len + 15) / 16;
     int part_blocks = P / 16;
     const int max_parts = ctx_blocks == 0 ? 1 : (ctx_blocks + part_blocks - 1) / part_blocks;

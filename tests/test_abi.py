@@ -52,14 +52,19 @@ def _dims(lib, **kw):
 
 
 def test_workspace_plan(lib):
+    # group 1 (CUDA-core kernel): automatic 512-token partitions
+    d1 = _dims(lib, num_heads=8)
+    assert lib.pa_decode_num_partitions(d1, 512, 0) == 1
+    assert lib.pa_decode_workspace_size(d1, 512, 0) == 0
+    assert lib.pa_decode_num_partitions(d1, 513, 0) == 2
+    assert lib.pa_decode_num_partitions(d1, 4096, 0) == 8
+    # group 4 at head_dim 128 (tensor-core kernel): automatic 1024-token partitions
     d = _dims(lib)
-    # short contexts fit one partition: no workspace
-    assert lib.pa_decode_num_partitions(d, 512, 0) == 1
-    assert lib.pa_decode_workspace_size(d, 512, 0) == 0
-    # automatic 512-token partitions above that
-    assert lib.pa_decode_num_partitions(d, 513, 0) == 2
-    assert lib.pa_decode_num_partitions(d, 4096, 0) == 8
-    ws = lib.pa_decode_workspace_size(d, 4096, 0)
+    assert lib.pa_decode_num_partitions(d, 1024, 0) == 1
+    assert lib.pa_decode_workspace_size(d, 1024, 0) == 0
+    assert lib.pa_decode_num_partitions(d, 1025, 0) == 2
+    assert lib.pa_decode_num_partitions(d, 4096, 0) == 4
+    ws = lib.pa_decode_workspace_size(d, 4096, 512)
     rows = 4 * 32 * 8
     assert ws >= rows * 128 * 4 + rows * 4
     # explicit partition sizes
@@ -89,37 +94,58 @@ def test_bad_partition_and_context(lib):
     assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), -1, 0) == -3
 
 
-def _decode_raw(lib, d, ptrs, nkv=8, maxlen=1000, part=0, ws=None, wsb=0):
+# The checks below hand the library fake device pointers and expect it to
+# reject every call on the host.  They run in a child process with no visible
+# GPU, so even a call that wrongly passed validation could not reach a device.
+HOST_CHECKS = r"""
+import ctypes, sys
+sys.path.insert(0, %(root)r)
+from paged_kv_cache_424_b200 import binding as lib
+
+def dims(**kw):
+    base = dict(num_seqs=4, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                max_blocks_per_seq=256, num_blocks=1024, dtype=lib.PA_BF16)
+    base.update(kw)
+    return lib.pa_dims(**base)
+
+def decode(d, ptrs, nkv=8, maxlen=2000, part=0, ws=None, wsb=0):
     out, q, k, v, bt, cl = ptrs
-    return lib.LIB.pa_decode(out, q, k, v, bt, cl, ctypes.c_float(0.1), nkv, ctypes.byref(d), maxlen, part, ws,
-                             wsb, None)
+    return lib.LIB.pa_decode(out, q, k, v, bt, cl, ctypes.c_float(0.1), nkv, ctypes.byref(d), maxlen, part,
+                             ws, wsb, None)
+
+d = dims()
+good = [ctypes.c_void_p(0x10000)] * 6
+assert decode(d, [None] + good[1:]) == -1
+assert decode(d, good, nkv=4) == -3
+assert decode(d, good) == -5                      # 2000 tokens: split, no workspace
+assert "workspace" in lib.pa_last_error()
+assert decode(d, good, ws=ctypes.c_void_p(0x20000), wsb=16) == -5
+assert decode(d, [ctypes.c_void_p(0x10008)] + good[1:], maxlen=100) == -7
+assert decode(dims(num_seqs=0), [None] * 6) == 0  # empty batch: nothing to do
+assert lib.LIB.pa_decode_noalloc(None, None, None, None, None, None, ctypes.c_float(0.1), 8,
+                                 ctypes.byref(d), 100, 0, None) == -1
+
+p = ctypes.c_void_p(0x10000)
+L = lib.LIB
+assert L.pa_reshape_and_cache(None, p, p, p, p, 4, ctypes.byref(d), None) == -1
+assert L.pa_reshape_and_cache(p, p, p, p, p, -1, ctypes.byref(d), None) == -3
+assert L.pa_reshape_and_cache(None, None, None, None, None, 0, ctypes.byref(d), None) == 0
+assert L.pa_reshape_and_cache(ctypes.c_void_p(0x10004), p, p, p, p, 4, ctypes.byref(d), None) == -7
+arr = (ctypes.c_void_p * 2)(0x10000, None)
+assert L.pa_copy_blocks(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p), 2, p, 3,
+                        ctypes.byref(d), None) == -1
+assert L.pa_copy_blocks(None, None, 0, None, 0, ctypes.byref(d), None) == 0
+assert L.pa_copy_blocks(None, None, 1, p, -1, ctypes.byref(d), None) == -3
+assert L.pa_device_error(None, None) == -1
+print("host checks ok")
+"""
 
 
-def test_decode_host_errors(lib):
-    d = _dims(lib)
-    good = [ctypes.c_void_p(0x10000)] * 6
-    assert _decode_raw(lib, d, [None] + good[1:]) == -1
-    assert _decode_raw(lib, d, good, nkv=4) == -3
-    assert _decode_raw(lib, d, good) == -5  # 1000 tokens -> 2 partitions, no workspace
-    assert "workspace" in lib.pa_last_error()
-    assert _decode_raw(lib, d, good, ws=ctypes.c_void_p(0x20000), wsb=16) == -5
-    bad = [ctypes.c_void_p(0x10008)] + good[1:]
-    assert _decode_raw(lib, d, bad, maxlen=100) == -7
-    d0 = _dims(lib, num_seqs=0)
-    assert _decode_raw(lib, d0, [None] * 6) == 0  # empty batch: nothing to do
-
-
-def test_cache_ops_host_errors(lib):
-    d = _dims(lib)
-    p = ctypes.c_void_p(0x10000)
-    L = lib.LIB
-    assert L.pa_reshape_and_cache(None, p, p, p, p, 4, ctypes.byref(d), None) == -1
-    assert L.pa_reshape_and_cache(p, p, p, p, p, -1, ctypes.byref(d), None) == -3
-    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, ctypes.byref(d), None) == 0
-    assert L.pa_reshape_and_cache(ctypes.c_void_p(0x10004), p, p, p, p, 4, ctypes.byref(d), None) == -7
-    arr = (ctypes.c_void_p * 2)(0x10000, None)
-    assert L.pa_copy_blocks(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p), 2, p, 3,
-                            ctypes.byref(d), None) == -1
-    assert L.pa_copy_blocks(None, None, 0, None, 0, ctypes.byref(d), None) == 0
-    assert L.pa_copy_blocks(None, None, 1, p, -1, ctypes.byref(d), None) == -3
-    assert L.pa_device_error(None, None) == -1
+def test_host_argument_errors(lib):
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", HOST_CHECKS % {"root": ROOT}], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "host checks ok" in r.stdout
