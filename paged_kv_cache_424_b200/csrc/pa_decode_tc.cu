@@ -9,18 +9,22 @@
 //   O^T (128 dims x 16)  = V^T (128 x 128 tokens) . P^T (128 x 16)  [PV]
 // (the G query rows padded to the MMA's N = 16).
 //
-// CTA = (512-token partition, KV head, sequence): 6 warps.
-//   warp 4  producer: per chunk, 2-D tiled TMA loads of the 8 blocks' K rows
-//           and V rows (16 rows x 64 dims per box, 128-byte swizzle) into the
-//           K tile and the V tile; blocks past the partition are loaded from
-//           an out-of-range row, which the TMA fills with zeros.
+// CTA = (partition, KV head, sequence): 7 warps.
+//   warp 4  K producer and warp 6  V producer: per chunk, 2-D tiled TMA loads
+//           of the 8 blocks' K (or V) rows (16 rows x 64 dims per box,
+//           128-byte swizzle) into the K (or V) tile, as soon as the previous
+//           chunk's MMA that read the tile has completed; blocks past the
+//           partition are loaded from an out-of-range row, which the TMA
+//           fills with zeros.  The partition's table slice is read once, 32
+//           entries per coalesced load.
 //   warp 5  MMA issuer (one thread): S into TMEM (double-buffered), then
 //           O = V^T P^T into TMEM (double-buffered), each completion signalled
 //           by tcgen05.commit on an mbarrier; allocates / frees TMEM.
 //   warps 0-3 softmax: thread t owns TMEM lane t = token t of S and output
 //           dim t of O.  Masks tokens past the context, keeps the online
-//           softmax with a lazy running max (raised only when a chunk's max
-//           beats it by 2^8), writes P (same 16-bit type as V) into a swizzled
+//           softmax with a lazy running max (raised only when some logit
+//           beats it by 2^8; a CTA-wide flag skips the max reduction in all
+//           other chunks), writes P (same 16-bit type as V) into a swizzled
 //           tile, and accumulates O chunk by chunk in registers.
 // Shared memory: K tile 32 KiB + V tile 32 KiB + Q 4 KiB + P 4 KiB (+ <1 KiB)
 // = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
@@ -42,7 +46,7 @@ constexpr int kD = 128;
 constexpr int kN = 16;              // MMA N: query heads padded to 16
 constexpr int kChunk = 128;         // tokens per chunk (MMA M)
 constexpr int kChunkBlocks = kChunk / kBlock;
-constexpr int kThreadsTc = 192;
+constexpr int kThreadsTc = 224;
 constexpr int kRegion = kChunk * 128;   // one 64-dim half of a K or V tile (bytes)
 
 // Shared-memory layout (bytes from the 1024-aligned base).
@@ -52,9 +56,9 @@ constexpr int kQOff = kVOff + 2 * kRegion;      // 65536
 constexpr int kPOff = kQOff + 2 * kN * 128;     // 69632
 constexpr int kRedOff = kPOff + 2 * kN * 128;   // 73728: [2][4][16] floats
 constexpr int kBarOff = kRedOff + 2 * 4 * kN * 4;
-constexpr int kNumBars = 9;
-constexpr int kMiscOff = kBarOff + kNumBars * 8;
-constexpr int kSmemTc = kMiscOff + 16;
+constexpr int kNumBars = 10;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;  // TMEM base, fail flag, 4 lazy-max flags
+constexpr int kSmemTc = kMiscOff + 32;
 
 // TMEM columns: S buffers at 0 and 16, O buffers at 32 and 48.
 constexpr uint32_t kTmemCols = 64;
@@ -77,12 +81,57 @@ __device__ __forceinline__ bool wait_ok(uint64_t *bar, uint32_t parity, int *fai
 
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// One producer warp streams one of the two tiles (K or V) chunk by chunk:
+// wait until the MMA that read the tile's previous chunk has completed
+// (`empty`), then load the chunk's 8 blocks (zeros past the partition).
+// The table slice is held in registers, 32 entries per window, the next
+// window prefetched one window ahead.
+__device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
+                                             uint64_t *full, uint64_t *empty, int *fail, int s, int kvh, int b0,
+                                             int nb, int nch, int oob_row, int lane) {
+    const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
+    auto window = [&](int w) -> int {
+        const int bi = w * 32 + lane;
+        return bi < nb ? (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock) : oob_row;
+    };
+    if (lane == 0) prefetch_tmap(tmap);
+    int cur = window(0);
+    int next = nb > 32 ? window(1) : oob_row;
+    for (int c = 0; c < nch; ++c) {
+        if (c > 0 && (c & 3) == 0) {
+            cur = next;
+            next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1) : oob_row;
+        }
+        const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
+        bool ok = true;
+        if (lane == 0) {
+            ok = c == 0 || wait_ok(empty, (c - 1) & 1, fail);
+            if (ok) mbar_arrive_expect_tx(full, 2 * kRegion);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane < kChunkBlocks) {
+            tc::tma_load_2d(tile + lane * 2048, tmap, 0, y, full);
+            tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 64, y, full);
+        }
+    }
+}
+
+// CTAs per SM: 3 (registers and shared memory both allow it) except for
+// groups of 16, whose per-thread state needs the registers of 2.
+__host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; }
+
 template <typename T, int G>
-__global__ void __launch_bounds__(kThreadsTc, 3)
+__global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
     using E = Elem<T>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr int kCols = G <= 8 ? 8 : 16;  // live TMEM columns of S and O
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *k_t = smem + kKOff;
     unsigned char *v_t = smem + kVOff;
@@ -91,9 +140,10 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
     float *red = reinterpret_cast<float *>(smem + kRedOff);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
     uint64_t *k_full = bars + 0, *k_empty = bars + 1, *v_full = bars + 2, *v_empty = bars + 3;
-    uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8;
+    uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8, *q_full = bars + 9;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMiscOff);
     int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
+    int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
 
     const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -128,6 +178,7 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
     }
     if (tid == 0) {
         *fail = 0;
+        for (int i = 0; i < 4; ++i) lazy_flag[i] = 0;
         mbar_init(k_full, 1);
         mbar_init(k_empty, 1);
         mbar_init(v_full, 1);
@@ -137,19 +188,8 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
         mbar_init(&o_full[0], 1);
         mbar_init(&o_full[1], 1);
         mbar_init(p_full, 128);
+        mbar_init(q_full, 128);
         fence_mbar_init();
-    }
-    if (tid < 128) {
-        // Q tile: rows = the group's query heads (zero rows up to 16), K-major
-        // 128-byte swizzle, two 64-dim regions.
-        const T *q = reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * kD;
-        for (int i = tid; i < kN * (kD / 8); i += 128) {
-            const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (r < G) v = *reinterpret_cast<const uint4 *>(q + r * kD + c16 * 8);
-            *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
-        }
-        fence_proxy_async_smem();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -157,34 +197,9 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 4) {
-        // ------------------------------ producer ------------------------------
-        const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
-        for (int c = 0; c < nch; ++c) {
-            const int bi = c * kChunkBlocks + lane;
-            int y = oob_row;
-            if (lane < kChunkBlocks && bi < nb) y = (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock);
-            bool ok = true;
-            if (lane == 0) {
-                ok = c == 0 || wait_ok(k_empty, (c - 1) & 1, fail);
-                if (ok) mbar_arrive_expect_tx(k_full, 2 * kRegion);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            if (lane < kChunkBlocks) {
-                tc::tma_load_2d(k_t + lane * 2048, &tmap_k, 0, y, k_full);
-                tc::tma_load_2d(k_t + kRegion + lane * 2048, &tmap_k, 64, y, k_full);
-            }
-            if (lane == 0) {
-                ok = c == 0 || wait_ok(v_empty, (c - 1) & 1, fail);
-                if (ok) mbar_arrive_expect_tx(v_full, 2 * kRegion);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            if (lane < kChunkBlocks) {
-                tc::tma_load_2d(v_t + lane * 2048, &tmap_v, 0, y, v_full);
-                tc::tma_load_2d(v_t + kRegion + lane * 2048, &tmap_v, 64, y, v_full);
-            }
-        }
+        produce_tile(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+    } else if (warp == 6) {
+        produce_tile(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
     } else if (warp == 5) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
@@ -204,7 +219,7 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
                 tc::commit(v_empty);
                 return true;
             };
-            bool ok = true;
+            bool ok = wait_ok(q_full, 0, fail);
             for (int c = 0; c < nch && ok; ++c) {
                 ok = wait_ok(k_full, c & 1, fail);
                 if (!ok) break;
@@ -224,6 +239,20 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
         __syncwarp();
     } else {
         // ------------------------------ softmax warps ------------------------------
+        {
+            // Q tile: rows = the group's query heads (zero rows up to 16),
+            // K-major 128-byte swizzle, two 64-dim regions.  Loaded while the
+            // producers already stream K and V.
+            const T *q = reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * kD;
+            for (int i = tid; i < kN * (kD / 8); i += 128) {
+                const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (r < G) v = *reinterpret_cast<const uint4 *>(q + r * kD + c16 * 8);
+                *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(q_full);
+        }
         const int t = tid;                                      // token of S, dim of O
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // TMEM lane quadrant
         float m[G], l[G], acc[G], alpha_prev[G];
@@ -237,8 +266,8 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
         auto epilogue = [&](int c) {
             if (!wait_ok(&o_full[c & 1], (c >> 1) & 1, fail)) return;
             tc::fence_after_sync();
-            float o[16];
-            tc::tmem_ld16(tmem + lane_base + o_col(c & 1), o);
+            float o[kCols];
+            tc::tmem_ld<kCols>(tmem + lane_base + o_col(c & 1), o);
 #pragma unroll
             for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha_prev[h], o[h]);
         };
@@ -248,37 +277,53 @@ __global__ void __launch_bounds__(kThreadsTc, 3)
             const int tok = tok0 + c * kChunk + t;
             const bool valid = tok < tok_end;
             bool ok = wait_ok(&s_full[c & 1], (c >> 1) & 1, fail);
+            bool exceed = false;
             if (ok) {
                 tc::fence_after_sync();
-                float sv[16];
-                tc::tmem_ld16(tmem + lane_base + s_col(c & 1), sv);
+                float sv[kCols];
+                tc::tmem_ld<kCols>(tmem + lane_base + s_col(c & 1), sv);
 #pragma unroll
-                for (int h = 0; h < G; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+                for (int h = 0; h < G; ++h) {
+                    x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+                    exceed |= x[h] > m[h] + kLazyMax;
+                }
             } else {
 #pragma unroll
                 for (int h = 0; h < G; ++h) x[h] = -INFINITY;
             }
-            // chunk max per head: warp max, then across the 4 warps
-            float *rc = red + (c & 1) * 4 * kN;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float v = x[h];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                if (lane == 0) rc[warp * kN + h] = v;
-            }
+            // Lazy running max: a CTA-wide flag says whether any logit of the
+            // chunk beats its head's running max by more than 2^8; only then
+            // are the per-head chunk maxima reduced and the state rescaled.
+            if (__any_sync(0xffffffffu, exceed) && lane == 0) lazy_flag[c & 3] = 1;
             softmax_sync();
+            const bool update = lazy_flag[c & 3] != 0;
+            if (t == 0) lazy_flag[(c + 2) & 3] = 0;  // slot of chunk c + 2: its readers are done
             float alpha[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) alpha[h] = 1.f;
+            if (update) {  // uniform across the 128 threads
+                float *rc = red + (c & 1) * 4 * kN;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float v = x[h];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    if (lane == 0) rc[warp * kN + h] = v;
+                }
+                softmax_sync();
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float cm = fmaxf(fmaxf(rc[h], rc[kN + h]), fmaxf(rc[2 * kN + h], rc[3 * kN + h]));
+                    if (cm > m[h] + kLazyMax) {
+                        alpha[h] = ex2(m[h] - cm);  // 0 on the first chunk (m = -inf)
+                        l[h] *= alpha[h];
+                        m[h] = cm;
+                    }
+                }
+            }
             T pv[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const float cm = fmaxf(fmaxf(rc[h], rc[kN + h]), fmaxf(rc[2 * kN + h], rc[3 * kN + h]));
-                alpha[h] = 1.f;
-                if (cm > m[h] + kLazyMax) {  // uniform across the 128 threads
-                    alpha[h] = ex2(m[h] - cm);
-                    l[h] *= alpha[h];
-                    m[h] = cm;
-                }
                 pv[h] = E::from_float(ex2(x[h] - m[h]));
                 l[h] += E::to_float(pv[h]);  // the rounded weight the MMA sees
             }
