@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256)
                              uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                              const int64_t *__restrict__ slot_mapping, int64_t num_items, int chunks_per_row,
                              int num_kv_heads, int64_t num_slots) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= num_items) return;
     const int64_t row = i / chunks_per_row;  // (token, kv head)
@@ -54,6 +56,8 @@ struct LayerPtrs {
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(const LayerPtrs ptrs, const int64_t *__restrict__ block_mapping, int64_t chunks_per_block,
                        int64_t num_blocks) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int pair = blockIdx.x, layer = blockIdx.y;
     const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
     if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -81,10 +85,10 @@ cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k
     const int64_t items = (int64_t)num_tokens * d.num_kv_heads * chunks;
     if (items == 0) return cudaSuccess;
     const int64_t grid = (items + 255) / 256;
-    reshape_and_cache_kernel<<<(unsigned)grid, 256, 0, stream>>>(
-        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), static_cast<uint4 *>(k_cache),
-        static_cast<uint4 *>(v_cache), slot_mapping, items, chunks, d.num_kv_heads, d.num_blocks * kBlock);
-    return cudaGetLastError();
+    return launch_pdl(reshape_and_cache_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
+                      static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), static_cast<uint4 *>(k_cache),
+                      static_cast<uint4 *>(v_cache), slot_mapping, items, chunks, (int)d.num_kv_heads,
+                      (int64_t)d.num_blocks * kBlock);
 }
 
 cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
@@ -99,8 +103,8 @@ cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int
             ptrs.k[i] = static_cast<uint4 *>(k_caches[l0 + i]);
             ptrs.v[i] = static_cast<uint4 *>(v_caches[l0 + i]);
         }
-        copy_blocks_kernel<<<dim3(num_pairs, nl), 256, 0, stream>>>(ptrs, block_mapping, chunks, d.num_blocks);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(copy_blocks_kernel, dim3(num_pairs, nl), dim3(256), 0, stream, ptrs, block_mapping,
+                                   chunks, (int64_t)d.num_blocks);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

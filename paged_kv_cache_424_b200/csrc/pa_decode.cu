@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     const int H = p.num_heads;
     const int head0 = kvh * G;
 
+    pdl_launch_dependents();
+    pdl_wait();
     const int L = checked_len(p, s, part_lmax(p), part == 0 && kvh == 0 && tid == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
@@ -184,6 +186,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
 template <typename T, int D>
 __global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p) {
     const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+    pdl_launch_dependents();
+    pdl_wait();
     const int L = checked_len(p, s, part_lmax(p), false);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
@@ -208,9 +212,7 @@ cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
     static int configured[kMaxDevices] = {};
     cudaError_t e = ensure_smem(kern, smem, configured);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.max_parts, p.num_kv_heads, p.num_seqs);
-    kern<<<grid, kWarps * 32, smem, stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(kWarps * 32), smem, stream, p);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, D, stream);
 }
@@ -231,14 +233,11 @@ cudaError_t launch_part_d(const DecodeParams &p, int group, cudaStream_t stream)
 
 cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream) {
     const dim3 grid(p.num_heads, p.num_seqs);
-    if (dtype == PA_F16) {
-        if (head_dim == 64) merge_part_kernel<__half, 64><<<grid, 64, 0, stream>>>(p);
-        else merge_part_kernel<__half, 128><<<grid, 128, 0, stream>>>(p);
-    } else {
-        if (head_dim == 64) merge_part_kernel<__nv_bfloat16, 64><<<grid, 64, 0, stream>>>(p);
-        else merge_part_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(p);
-    }
-    return cudaGetLastError();
+    if (dtype == PA_F16)
+        return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, dim3(64), 0, stream, p)
+                              : launch_pdl(merge_part_kernel<__half, 128>, grid, dim3(128), 0, stream, p);
+    return head_dim == 64 ? launch_pdl(merge_part_kernel<__nv_bfloat16, 64>, grid, dim3(64), 0, stream, p)
+                          : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p);
 }
 
 cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group,

@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     const int H = p.num_heads, head0 = kvh * G;
     T *out = reinterpret_cast<T *>(p.out);
 
+    pdl_launch_dependents();
+    pdl_wait();
     const int L = checked_len(p, s, part_lmax_tc(p), part == 0 && kvh == 0 && tid == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
@@ -443,9 +445,8 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     }
     e = ensure_smem(kern, kSmemTc, configured);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.max_parts, p.num_kv_heads, p.num_seqs);
-    kern<<<grid, kThreadsTc, kSmemTc, stream>>>(p, tk, tv, (int)rows);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(kThreadsTc), kSmemTc, stream, p, tk, tv,
+                   (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
 }
