@@ -48,7 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha7b", choices=["tiny", "mha7b", "gqa8b", "long70b", "cow"])
+    ap.add_argument("--workload", default="mha7b", choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "swap"],
+                    help="decode scenario, or 'swap' for pa_swap_blocks device <-> pinned host throughput")
     ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
     ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
@@ -447,9 +448,70 @@ def run_reference(args):
     }), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# swap_blocks: device <-> page-locked host block copies (preemption)
+# ---------------------------------------------------------------------------
+def run_swap(args):
+    """Swap 2048 blocks of the 7B shape (32 KV heads x 16 x 128 fp16: 128 KiB
+    of K and 128 KiB of V each) out to a pinned host pool and back in.  One
+    step = one swap-out + one swap-in; value = GB/s moved per direction."""
+    import torch
+    from paged_kv_cache_424_b200 import build
+    build.build()
+    from paged_kv_cache_424_b200 import binding as pa
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    nb_dev, nb_host, pairs, shape = 8192, 4096, 2048, (32, 16, 128)
+    rng = np.random.default_rng(7 + rank)
+    dk = torch.randn((nb_dev, *shape), device=dev, dtype=torch.float16)
+    dv = torch.randn((nb_dev, *shape), device=dev, dtype=torch.float16)
+    hk = torch.empty((nb_host, *shape), dtype=torch.float16).pin_memory()
+    hv = torch.empty((nb_host, *shape), dtype=torch.float16).pin_memory()
+    out_map = torch.from_numpy(np.stack([rng.choice(nb_dev, pairs, replace=False),
+                                         rng.choice(nb_host, pairs, replace=False)], 1).astype(np.int64)).to(dev)
+    in_map = torch.stack([out_map[:, 1], out_map[:, 0]], 1).contiguous()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        pa.pa_swap_blocks(dk, dv, hk, hv, out_map, stream=stream)
+        pa.pa_swap_blocks(hk, hv, dk, dv, in_map, stream=stream)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    barrier(world)
+    e[0].record(stream)
+    for _ in range(K):
+        pa.pa_swap_blocks(dk, dv, hk, hv, out_map, stream=stream)
+    e[1].record(stream)
+    for _ in range(K):
+        pa.pa_swap_blocks(hk, hv, dk, dv, in_map, stream=stream)
+    e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    out_ms = max_over_ranks(e[0].elapsed_time(e[1]) / K, world, dev)
+    in_ms = max_over_ranks(e[1].elapsed_time(e[2]) / K, world, dev)
+    if pa.pa_device_error(stream) != 0:
+        raise SystemExit("device error word set")
+    nbytes = pairs * 2 * int(np.prod(shape)) * 2
+    if rank == 0:
+        print(json.dumps({
+            "metric": "pa_swap_blocks throughput, device <-> page-locked host (GB/s per direction)",
+            "value": nbytes * world / ((out_ms + in_ms) / 2 / 1e3) / 1e9, "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": out_ms + in_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": f"swap {pairs} blocks of 32x16x128 fp16 K+V ({nbytes / 2**20:.0f} MiB) "
+                                   f"out of a {nb_dev}-block device pool and back in",
+                       "swap_out_gbs": nbytes / (out_ms / 1e3) / 1e9, "swap_in_gbs": nbytes / (in_ms / 1e3) / 1e9},
+            "gpu_launches": 2 * K}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.workload == "swap":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "swap throughput has no CPU-oracle arm"}))
+            return
+        run_swap(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

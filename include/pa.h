@@ -6,6 +6,7 @@
  *
  *   pa_reshape_and_cache  write each new token's key/value into its slot
  *   pa_copy_blocks        copy-on-write duplication of shared blocks
+ *   pa_swap_blocks        block copies between device and host pools (preemption)
  *   pa_decode             single-query attention of every sequence over its
  *                         cached tokens, gathered through its block table
  *
@@ -64,7 +65,8 @@ typedef enum pa_status {
     PA_ERR_UNSUPPORTED = -4, /* block_size / head_dim / group size not built */
     PA_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
     PA_ERR_CUDA = -6,        /* a CUDA launch or query failed */
-    PA_ERR_ALIGN = -7        /* a data pointer is not 16-byte aligned */
+    PA_ERR_ALIGN = -7,       /* a data pointer is not 16-byte aligned */
+    PA_ERR_MEMORY = -8       /* a pointer the device cannot address (pageable host memory) */
 } pa_status;
 
 typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
@@ -188,6 +190,29 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
 pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
                          const int64_t *block_mapping, int32_t num_pairs, const pa_dims *dims,
                          void *stream);
+
+/*
+ * Swap blocks between two pools ("vLLM PagedAttention 大模型推理架构深度实战"
+ * section 3.2: under memory pressure a low-priority sequence's KV cache is
+ * swapped out to CPU memory and resumed later; section 九 item 5: swapped-out
+ * KV kept in fast host memory).  For every pair i < num_pairs,
+ * (src, dst) = block_mapping[i]:
+ *     dst_k[dst] = src_k[src],   dst_v[dst] = src_v[src]
+ * (all num_kv_heads * 16 * head_dim elements of a block; dims gives the block
+ * geometry and dtype, dims->num_blocks is not used).  The source pools hold
+ * src_num_blocks blocks, the destination pools dst_num_blocks.  Each pool may
+ * be device memory or page-locked host memory the device can address with
+ * the same pointer (cudaHostAlloc / cudaHostRegister under unified
+ * addressing): device -> host swaps out, host -> device swaps in.
+ * block_mapping [num_pairs, 2] int64 is device or page-locked host memory.
+ * Every pointer is checked on the host (cudaPointerGetAttributes): pageable
+ * host memory is refused with PA_ERR_MEMORY before anything is enqueued.
+ * One kernel moves every pair; destinations must be distinct.  Bit-exact.
+ * Out-of-range ids are skipped and flagged (PA_DEVERR_COPY_PAIR).
+ */
+pa_status pa_swap_blocks(const void *src_k, const void *src_v, int64_t src_num_blocks, void *dst_k,
+                         void *dst_v, int64_t dst_num_blocks, const int64_t *block_mapping,
+                         int32_t num_pairs, const pa_dims *dims, void *stream);
 
 /* Thread-local description of the last non-OK status returned on this
  * thread ("" if none).  Owned by the library; valid until the next call. */

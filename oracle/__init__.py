@@ -75,6 +75,8 @@ class Oracle:
         lib.oracle_reshape_and_cache.restype = ctypes.c_int
         lib.oracle_copy_blocks.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, i64]
         lib.oracle_copy_blocks.restype = ctypes.c_int
+        lib.oracle_swap_blocks.argtypes = [vp, vp, i64, vp, vp, i64, vp, i32, i32, i32, i32]
+        lib.oracle_swap_blocks.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -147,6 +149,20 @@ class Oracle:
                                           L, _p(bm), bm.shape[0], Hk, D, B, NB)
         if rc != 0:
             raise OracleError(f"oracle_copy_blocks returned {rc}")
+
+    def swap_blocks(self, dst_k, dst_v, src_k, src_v, block_mapping) -> None:
+        """In place: block dst of the destination pools becomes a copy of block
+        src of the source pools (K and V)."""
+        bm = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+        NBd, Hk, B, D = dst_k.shape
+        NBs = src_k.shape[0]
+        for a, nb in ((dst_k, NBd), (dst_v, NBd), (src_k, NBs), (src_v, NBs)):
+            if a.shape != (nb, Hk, B, D) or a.dtype != np.uint16 or not a.flags.c_contiguous:
+                raise OracleError("pools must be C-contiguous uint16 with matching block shapes")
+        rc = self._lib.oracle_swap_blocks(_p(dst_k), _p(dst_v), NBd, _p(src_k), _p(src_v), NBs, _p(bm),
+                                          bm.shape[0], Hk, D, B)
+        if rc != 0:
+            raise OracleError(f"oracle_swap_blocks returned {rc}")
 
 
 def paged_decode(*args, **kw):

@@ -26,6 +26,10 @@
  *  - ybb.press section 六 "架构总览" (decode loop): each iteration writes the
  *    new token's K/V into its KV-cache block; reshape_and_cache is the plain
  *    indexed assignment.
+ *  - ybb.press section 3.2 (preemption: a sequence's KV cache is swapped out
+ *    to CPU memory and resumed later) and section 九 item 5 (swapped-out KV
+ *    kept in fast host memory): swap_blocks is a block copy between two
+ *    pools.
  *
  * Layouts (row-major, contiguous; element = 16-bit fp16 or bf16 bit pattern):
  *   q, out        [num_seqs, num_heads, head_dim]   (out is double here)
@@ -252,6 +256,28 @@ int oracle_copy_blocks(uint16_t *const *k_caches, uint16_t *const *v_caches, int
             memmove(k_caches[l] + dst * elems, k_caches[l] + src * elems, sizeof(uint16_t) * elems);
             memmove(v_caches[l] + dst * elems, v_caches[l] + src * elems, sizeof(uint16_t) * elems);
         }
+    }
+    return ORC_OK;
+}
+
+/*
+ * Swap between two pools: for every pair (src, dst), block dst of the
+ * destination K and V pools becomes a copy of block src of the source pools.
+ */
+int oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, int64_t dst_num_blocks, const uint16_t *src_k,
+                       const uint16_t *src_v, int64_t src_num_blocks, const int64_t *block_mapping,
+                       int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0) return ORC_ERR_ARG;
+    if (num_pairs > 0 && (!dst_k || !dst_v || !src_k || !src_v || !block_mapping)) return ORC_ERR_ARG;
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return ORC_ERR_RANGE;
+    }
+    const int64_t elems = (int64_t)num_kv_heads * block_size * head_dim;
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
+        memcpy(dst_k + dst * elems, src_k + src * elems, sizeof(uint16_t) * elems);
+        memcpy(dst_v + dst * elems, src_v + src * elems, sizeof(uint16_t) * elems);
     }
     return ORC_OK;
 }

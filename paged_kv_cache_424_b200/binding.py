@@ -20,14 +20,14 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_OK = 0
 STATUS = {0: "PA_OK", -1: "PA_ERR_NULL", -2: "PA_ERR_DTYPE", -3: "PA_ERR_SHAPE", -4: "PA_ERR_UNSUPPORTED",
-          -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_CUDA", -7: "PA_ERR_ALIGN"}
+          -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_CUDA", -7: "PA_ERR_ALIGN", -8: "PA_ERR_MEMORY"}
 PA_F16, PA_BF16 = 0, 1
 DEVERR = {1: "BLOCK_ID", 2: "CONTEXT", 4: "SLOT", 8: "COPY_PAIR", 16: "TIMEOUT"}
 
 # The C entry points declared in include/pa.h, in declaration order.
 EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_decode_noalloc",
            "pa_reshape_and_cache",
-           "pa_copy_blocks", "pa_last_error", "pa_device_error", "pa_version"]
+           "pa_copy_blocks", "pa_swap_blocks", "pa_last_error", "pa_device_error", "pa_version"]
 
 
 class LibraryMissing(RuntimeError):
@@ -64,6 +64,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
     lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_swap_blocks.argtypes = [vp, vp, i64, vp, vp, i64, vp, i32, dp, vp]
+    lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_last_error.argtypes = []
     lib.pa_last_error.restype = ctypes.c_char_p
     lib.pa_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -215,6 +217,24 @@ def pa_copy_blocks(k_caches: Sequence[torch.Tensor], v_caches: Sequence[torch.Te
     pairs = block_mapping.numel() // 2
     st = LIB.pa_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), L,
                             _ptr(block_mapping), int(pairs), ctypes.byref(dims), _stream(stream))
+    _check(st)
+
+
+def pa_swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, dst_v: torch.Tensor,
+                   block_mapping: torch.Tensor, stream=None) -> None:
+    """Block dst of the destination pools becomes a copy of block src of the
+    source pools; each pool a CUDA tensor or a pinned CPU tensor."""
+    for t in (src_k, src_v, dst_k, dst_v, block_mapping):
+        if not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+            raise ValueError("pools and mapping must be contiguous CUDA tensors or pinned CPU tensors")
+    if block_mapping.dtype != torch.int64:
+        raise TypeError("block_mapping must be int64")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_v.shape != src_k.shape or dst_v.shape != dst_k.shape:
+        raise ValueError("pools disagree on the block shape")
+    dims = cache_dims(src_k)
+    st = LIB.pa_swap_blocks(_ptr(src_k), _ptr(src_v), int(src_k.shape[0]), _ptr(dst_k), _ptr(dst_v),
+                            int(dst_k.shape[0]), _ptr(block_mapping), int(block_mapping.numel() // 2),
+                            ctypes.byref(dims), _stream(stream))
     _check(st)
 
 

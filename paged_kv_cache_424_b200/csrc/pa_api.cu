@@ -206,6 +206,45 @@ pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t n
     return PA_OK;
 }
 
+// The address the device uses for `p`: itself for device / managed memory,
+// the mapped address for page-locked host memory; nullptr when the device
+// cannot address it (pageable host memory).
+const void *device_address(const void *p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+    if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+    return nullptr;
+}
+
+pa_status pa_swap_blocks(const void *src_k, const void *src_v, int64_t src_num_blocks, void *dst_k, void *dst_v,
+                         int64_t dst_num_blocks, const int64_t *block_mapping, int32_t num_pairs, const pa_dims *dims,
+                         void *stream) {
+    pa_status st = check_dims(dims, false);
+    if (st != PA_OK) return st;
+    if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0)
+        return fail(PA_ERR_SHAPE, "num_pairs must be >= 0 and both pools must have blocks");
+    if (num_pairs == 0) return PA_OK;
+    if (num_pairs > 65535) return fail(PA_ERR_SHAPE, "num_pairs %d > 65535", num_pairs);
+    if (!src_k || !src_v || !dst_k || !dst_v || !block_mapping) return fail(PA_ERR_NULL, "a required pointer is NULL");
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v))
+        return fail(PA_ERR_ALIGN, "pools must be 16-byte aligned");
+    const void *sk = device_address(src_k), *sv = device_address(src_v);
+    const void *dk = device_address(dst_k), *dv = device_address(dst_v);
+    const void *bm = device_address(block_mapping);
+    if (!sk || !sv || !dk || !dv || !bm)
+        return fail(PA_ERR_MEMORY, "a pool or the mapping is not device or page-locked host memory");
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    cudaError_t e = pa::launch_swap_blocks(sk, sv, src_num_blocks, const_cast<void *>(dk), const_cast<void *>(dv),
+                                           dst_num_blocks, static_cast<const int64_t *>(bm), num_pairs, cd,
+                                           static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_swap_blocks launch");
+    return PA_OK;
+}
+
 pa_status pa_device_error(void *stream, uint32_t *word) {
     if (!word) return fail(PA_ERR_NULL, "word is NULL");
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -6,6 +6,11 @@
 //   pool [NB, Hk, 16, D].
 // copy_blocks: same page, section 2.3: a block shared by several sequences is
 //   copied before one of them writes into it (copy-on-write).
+// swap_blocks: same page, section 3.2 (a preempted sequence's KV cache is
+//   swapped out to CPU memory and swapped back in on resume) and section 九
+//   item 5 (swapped-out KV kept in fast host memory): block copies between a
+//   device pool and a page-locked host pool, which the kernel reads or writes
+//   directly through unified addressing (one launch for all pairs).
 //
 // Both are pure data movement (bit-exact) and HBM-bound: 16-byte vector
 // loads and stores, consecutive threads on consecutive 16-byte chunks.
@@ -76,7 +81,50 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// CTA = (pair, K or V): copies one block between the two pools.  Each thread
+// keeps 4 16-byte loads in flight before storing, since host-side accesses
+// cross the PCIe / chip-to-chip link with a long latency.
+__global__ void __launch_bounds__(256)
+    swap_blocks_kernel(const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v, int64_t src_blocks,
+                       uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v, int64_t dst_blocks,
+                       const int64_t *__restrict__ block_mapping, int64_t chunks_per_block) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int pair = blockIdx.x;
+    const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(PA_DEVERR_COPY_PAIR);
+        return;
+    }
+    const uint4 *s = (blockIdx.y == 0 ? src_k : src_v) + src * chunks_per_block;
+    uint4 *d = (blockIdx.y == 0 ? dst_k : dst_v) + dst * chunks_per_block;
+    constexpr int kUnroll = 4;
+    for (int64_t i0 = threadIdx.x; i0 < chunks_per_block; i0 += (int64_t)blockDim.x * kUnroll) {
+        uint4 r[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = i0 + (int64_t)u * blockDim.x;
+            if (i < chunks_per_block) r[u] = s[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = i0 + (int64_t)u * blockDim.x;
+            if (i < chunks_per_block) d[i] = r[u];
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_swap_blocks(const void *src_k, const void *src_v, int64_t src_blocks, void *dst_k, void *dst_v,
+                               int64_t dst_blocks, const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
+                               cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim / 8;
+    return launch_pdl(swap_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream, static_cast<const uint4 *>(src_k),
+                      static_cast<const uint4 *>(src_v), src_blocks, static_cast<uint4 *>(dst_k),
+                      static_cast<uint4 *>(dst_v), dst_blocks, block_mapping, chunks);
+}
 
 cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
                                      const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,

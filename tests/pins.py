@@ -392,6 +392,31 @@ def pin_copy_on_write_keeps_sharers(orc):
     assert np.array_equal(kc[3, :, 10], key[0]), "the writer's token is missing"
 
 
+def pin_swap_blocks_matches_slices(orc):
+    """Swap out to a second (host) pool and back: numpy slice copies, and a
+    round trip restores the original blocks."""
+    rng = np.random.default_rng(16)
+    Hk, B, D = 2, 16, 8
+    dev_k = rand_bits(rng, (9, Hk, B, D), "bf16")
+    dev_v = rand_bits(rng, (9, Hk, B, D), "bf16")
+    host_k = np.zeros((5, Hk, B, D), np.uint16)
+    host_v = np.zeros((5, Hk, B, D), np.uint16)
+    out_map = np.array([[7, 0], [2, 3], [4, 1]], dtype=np.int64)
+    want_k = host_k.copy()
+    want_v = host_v.copy()
+    want_k[out_map[:, 1]] = dev_k[out_map[:, 0]]
+    want_v[out_map[:, 1]] = dev_v[out_map[:, 0]]
+    orc.swap_blocks(host_k, host_v, dev_k, dev_v, out_map)
+    assert np.array_equal(host_k, want_k) and np.array_equal(host_v, want_v), "swap-out differs"
+    back = np.stack([out_map[:, 1], [0, 5, 6]], axis=1)
+    orig_k, orig_v = dev_k.copy(), dev_v.copy()
+    orc.swap_blocks(dev_k, dev_v, host_k, host_v, back)
+    assert np.array_equal(dev_k[[0, 5, 6]], orig_k[[7, 2, 4]]), "swap-in did not restore the blocks"
+    assert np.array_equal(dev_v[[0, 5, 6]], orig_v[[7, 2, 4]]), "swap-in did not restore the blocks"
+    keep = [1, 3, 7, 8]
+    assert np.array_equal(dev_k[keep], orig_k[keep]), "swap-in touched other blocks"
+
+
 def pin_brute_force_tiny(orc):
     """The first scenario (4 seqs, lengths 1/17/33/100) against the pure
     Python brute force, every (sequence, head)."""

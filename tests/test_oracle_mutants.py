@@ -44,6 +44,8 @@ MUTANTS = {
                     ""),
     "copy_reversed": ("memmove(k_caches[l] + dst * elems, k_caches[l] + src * elems",
                       "memmove(k_caches[l] + src * elems, k_caches[l] + dst * elems"),
+    "swap_only_k": ("memcpy(dst_v + dst * elems, src_v + src * elems, sizeof(uint16_t) * elems);", ""),
+    "swap_direction": ("memcpy(dst_k + dst * elems, src_k + src * elems", "memcpy(dst_k + src * elems, src_k + dst * elems"),
     "zero_length_not_zeroed": ("for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;\n        if (n == 0) continue;",
                                "if (n == 0) { o[0] = 1.0; continue; }\n        "
                                "for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;"),
