@@ -77,6 +77,16 @@ class Oracle:
         lib.oracle_copy_blocks.restype = ctypes.c_int
         lib.oracle_swap_blocks.argtypes = [vp, vp, i64, vp, vp, i64, vp, i32, i32, i32, i32]
         lib.oracle_swap_blocks.restype = ctypes.c_int
+        lib.oracle_paged_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, dbl, dbl, dbl, i32, i32, i32, i32, i32,
+                                                 i32, i64, i32]
+        lib.oracle_paged_decode_fp8.restype = ctypes.c_int
+        lib.oracle_reshape_and_cache_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32,
+                                                     ctypes.c_float, ctypes.c_float]
+        lib.oracle_reshape_and_cache_fp8.restype = ctypes.c_int
+        lib.oracle_quantize_e4m3_n.argtypes = [vp, vp, i64]
+        lib.oracle_quantize_e4m3_n.restype = None
+        lib.oracle_widen_e4m3_n.argtypes = [vp, vp, i64]
+        lib.oracle_widen_e4m3_n.restype = None
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -163,6 +173,59 @@ class Oracle:
                                           bm.shape[0], Hk, D, B)
         if rc != 0:
             raise OracleError(f"oracle_swap_blocks returned {rc}")
+
+    # -- FP8 E4M3 KV cache ---------------------------------------------------
+    def quantize_e4m3(self, y) -> np.ndarray:
+        """float32 values -> E4M3 codes (nearest, ties to even, clamped to 448)."""
+        y = np.ascontiguousarray(y, dtype=np.float32)
+        out = np.empty(y.shape, dtype=np.uint8)
+        self._lib.oracle_quantize_e4m3_n(_p(out), _p(y), y.size)
+        return out
+
+    def widen_e4m3(self, c) -> np.ndarray:
+        c = np.ascontiguousarray(c, dtype=np.uint8)
+        out = np.empty(c.shape, dtype=np.float64)
+        self._lib.oracle_widen_e4m3_n(_p(out), _p(c), c.size)
+        return out
+
+    def paged_decode_fp8(self, q, k_cache, v_cache, block_tables, context_lens, scale: float, k_scale: float,
+                         v_scale: float, dtype: str) -> np.ndarray:
+        """paged_decode over E4M3 caches: K = decode(code) * k_scale, V likewise."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        k_cache = np.ascontiguousarray(k_cache, dtype=np.uint8)
+        v_cache = np.ascontiguousarray(v_cache, dtype=np.uint8)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, H, D = q.shape
+        NB, Hk, B, D2 = k_cache.shape
+        if D2 != D or v_cache.shape != k_cache.shape or bt.shape[0] != S or cl.shape != (S,):
+            raise OracleError("shape mismatch")
+        MB = bt.shape[1] if bt.ndim == 2 else 0
+        out = np.zeros((S, H, D), dtype=np.float64)
+        rc = self._lib.oracle_paged_decode_fp8(_p(out), _p(q), _p(k_cache), _p(v_cache), _p(bt), _p(cl),
+                                               float(scale), float(k_scale), float(v_scale), S, H, Hk, D, B, MB,
+                                               NB, _DTYPE_CODE[dtype])
+        if rc != 0:
+            raise OracleError(f"oracle_paged_decode_fp8 returned {rc}")
+        return out
+
+    def reshape_and_cache_fp8(self, k_cache, v_cache, key, value, slot_mapping, dtype: str, k_scale: float,
+                              v_scale: float) -> None:
+        """In place: E4M3 codes of key[t] / k_scale (value[t] / v_scale) into slot[t]."""
+        for a in (k_cache, v_cache):
+            if a.dtype != np.uint8 or not a.flags.c_contiguous:
+                raise OracleError("FP8 caches must be C-contiguous uint8")
+        key = np.ascontiguousarray(key, dtype=np.uint16)
+        value = np.ascontiguousarray(value, dtype=np.uint16)
+        sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        NB, Hk, B, D = k_cache.shape
+        T = sm.shape[0]
+        if key.shape != (T, Hk, D) or value.shape != (T, Hk, D):
+            raise OracleError("key/value shape mismatch")
+        rc = self._lib.oracle_reshape_and_cache_fp8(_p(k_cache), _p(v_cache), _p(key), _p(value), _p(sm), T, Hk,
+                                                    D, B, NB, _DTYPE_CODE[dtype], float(k_scale), float(v_scale))
+        if rc != 0:
+            raise OracleError(f"oracle_reshape_and_cache_fp8 returned {rc}")
 
 
 def paged_decode(*args, **kw):

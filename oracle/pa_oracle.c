@@ -41,6 +41,15 @@
  *                 negative = skip
  *   block_mapping [num_pairs, 2] int64 (src, dst)
  *
+ * FP8 KV cache (a later variant of the same path; the pages name FP8 only
+ * for weights, ybb.press section 5.2, and KV-cache compression as a goal,
+ * section 九 item 3): caches of OCP FP8 E4M3 codes (bias 7, 3 mantissa
+ * bits, no infinities, S.1111.111 = NaN, largest finite 448) with one fp32
+ * scale per tensor: element = decode(code) * scale.  Quantisation of a
+ * 16-bit value x: y = float(x) / scale in IEEE fp32 (one correctly rounded
+ * division), then the E4M3 value nearest to y, ties to the even code,
+ * magnitudes beyond 448 clamped to 448 ("saturate to finite"), NaN -> NaN.
+ *
  * Readings where the pages are silent: query head h reads KV head
  * h / (num_heads / num_kv_heads) (contiguous GQA groups); a context length of
  * zero yields an all-zero output row.
@@ -87,6 +96,47 @@ static double widen_bf16(uint16_t h) {
 
 static double widen(uint16_t h, int32_t dtype) {
     return dtype == ORC_BF16 ? widen_bf16(h) : widen_f16(h);
+}
+
+/* OCP FP8 E4M3 code -> double: sign, 4-bit exponent (bias 7), 3-bit
+ * fraction; exponent 0 is subnormal (fraction * 2^-9); code S.1111.111 is
+ * NaN (there are no infinities). */
+static double widen_e4m3(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xf;
+    int m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(m + 8), e - 10);
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to y (ties to the even code), clamped to +-448. */
+static uint8_t quantize_e4m3(float y) {
+    if (y != y) return 0x7f;
+    double a = fabs((double)y);
+    uint8_t best = 0;
+    double best_err = a;  /* code 0 = +0 */
+    for (uint8_t c = 1; c < 0x7f; ++c) {  /* every positive finite code, ascending */
+        double err = fabs(widen_e4m3(c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    if (a > 448.0) best = 0x7e;  /* saturate to finite */
+    return (uint8_t)(best | (y < 0 ? 0x80 : 0));
+}
+
+void oracle_quantize_e4m3_n(uint8_t *out, const float *y, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = quantize_e4m3(y[i]);
+}
+void oracle_widen_e4m3_n(double *out, const uint8_t *c, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = widen_e4m3(c[i]);
 }
 
 int oracle_set_num_threads(int n) {
@@ -278,6 +328,103 @@ int oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, int64_t dst_num_blocks,
         int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
         memcpy(dst_k + dst * elems, src_k + src * elems, sizeof(uint16_t) * elems);
         memcpy(dst_v + dst * elems, src_v + src * elems, sizeof(uint16_t) * elems);
+    }
+    return ORC_OK;
+}
+
+/*
+ * Decode attention over FP8 E4M3 caches with per-tensor scales: the same
+ * definition as oracle_paged_decode, with K_s[j, d] = decode(k_code) * k_scale
+ * and V_s[j, d] = decode(v_code) * v_scale; q and out as before (q_dtype).
+ */
+int oracle_paged_decode_fp8(double *out, const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                            const int32_t *block_tables, const int32_t *context_lens, double scale,
+                            double k_scale, double v_scale, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t max_blocks_per_seq, int64_t num_blocks, int32_t q_dtype) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return ORC_ERR_ARG;
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq < 0 || num_blocks <= 0 || num_heads % num_kv_heads != 0)
+        return ORC_ERR_ARG;
+    if (q_dtype != ORC_F16 && q_dtype != ORC_BF16) return ORC_ERR_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t n = context_lens[s];
+        if (n < 0 || (int64_t)n > (int64_t)max_blocks_per_seq * block_size) return ORC_ERR_RANGE;
+        for (int32_t i = 0; i < (n + block_size - 1) / block_size; ++i) {
+            int32_t b = block_tables[(int64_t)s * max_blocks_per_seq + i];
+            if (b < 0 || (int64_t)b >= num_blocks) return ORC_ERR_RANGE;
+        }
+    }
+    const int32_t group = num_heads / num_kv_heads;
+    const int64_t pairs = (int64_t)num_seqs * num_heads;
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < pairs; ++p) {
+        const int32_t s = (int32_t)(p / num_heads), h = (int32_t)(p % num_heads);
+        const int32_t kvh = h / group, n = context_lens[s];
+        double *o = out + p * head_dim;
+        for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+        if (n == 0) continue;
+        double *x = (double *)malloc(sizeof(double) * (size_t)n);
+        if (!x) {
+#pragma omp atomic write
+            status = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int32_t j = 0; j < n; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double dot = 0.0;
+            for (int32_t d = 0; d < head_dim; ++d)
+                dot += widen(q[p * head_dim + d], q_dtype) * (widen_e4m3(k_cache[row + d]) * k_scale);
+            x[j] = scale * dot;
+        }
+        double m = x[0];
+        for (int32_t j = 1; j < n; ++j)
+            if (x[j] > m) m = x[j];
+        double z = 0.0;
+        for (int32_t j = 0; j < n; ++j) {
+            x[j] = exp(x[j] - m);
+            z += x[j];
+        }
+        for (int32_t j = 0; j < n; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double w = x[j] / z;
+            for (int32_t d = 0; d < head_dim; ++d) o[d] += w * (widen_e4m3(v_cache[row + d]) * v_scale);
+        }
+        free(x);
+    }
+    return status;
+}
+
+/*
+ * Cache write into FP8 E4M3 caches: for every token t with slot >= 0,
+ *   k_cache[slot / block_size, h, slot % block_size, d] =
+ *       quantize(float(key[t, h, d]) / k_scale)      (same for value, v_scale)
+ */
+int oracle_reshape_and_cache_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint16_t *key, const uint16_t *value,
+                                 const int64_t *slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t block_size, int64_t num_blocks, int32_t dtype,
+                                 float k_scale, float v_scale) {
+    if (!k_cache || !v_cache || (num_tokens > 0 && (!key || !value || !slot_mapping))) return ORC_ERR_ARG;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return ORC_ERR_ARG;
+    if (dtype != ORC_F16 && dtype != ORC_BF16) return ORC_ERR_ARG;
+    for (int32_t t = 0; t < num_tokens; ++t)
+        if (slot_mapping[t] >= 0 && slot_mapping[t] / block_size >= num_blocks) return ORC_ERR_RANGE;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                k_cache[dst + d] = quantize_e4m3((float)widen(key[src + d], dtype) / k_scale);
+                v_cache[dst + d] = quantize_e4m3((float)widen(value[src + d], dtype) / v_scale);
+            }
+        }
     }
     return ORC_OK;
 }

@@ -417,6 +417,86 @@ def pin_swap_blocks_matches_slices(orc):
     assert np.array_equal(dev_k[keep], orig_k[keep]), "swap-in touched other blocks"
 
 
+# ---------------------------------------------------------------------------
+# FP8 E4M3 KV-cache pins
+# ---------------------------------------------------------------------------
+def e4m3_torch(codes) -> np.ndarray:
+    """torch's own E4M3 decoding (a library routine)."""
+    t = torch.from_numpy(np.asarray(codes, dtype=np.uint8).copy()).view(torch.float8_e4m3fn)
+    return t.float().numpy().astype(np.float64)
+
+
+def pin_e4m3_widen_every_code(orc):
+    codes = np.arange(256, dtype=np.uint8)
+    got, want = orc.widen_e4m3(codes), e4m3_torch(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want)), "NaN codes differ"
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok]), "E4M3 decoding differs from torch"
+
+
+def pin_e4m3_quantize_matches_torch_in_range(orc):
+    """Random values, every representable value and every midpoint between
+    neighbours (the tie cases) up to 448: same codes as torch's
+    round-to-nearest-even conversion."""
+    rng = np.random.default_rng(17)
+    vals = e4m3_torch(np.arange(0, 0x7f, dtype=np.uint8))        # +0 .. 448
+    mids = (vals[:-1] + vals[1:]) / 2
+    y = np.concatenate([vals, mids, rng.uniform(-448, 448, 4000), rng.uniform(-1, 1, 4000),
+                        rng.uniform(-2 ** -6, 2 ** -6, 2000)]).astype(np.float32)
+    y = np.concatenate([y, -y])
+    want = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = orc.quantize_e4m3(y)
+    zero = y == 0  # torch keeps the sign of zero; compare -0 and +0 by value
+    assert np.array_equal(got[~zero], want[~zero]), "quantisation differs from torch in range"
+    assert np.all(orc.widen_e4m3(got[zero]) == 0)
+
+
+def pin_e4m3_saturates_to_finite(orc):
+    y = np.array([448.5, 463.9, 464.0, 500.0, 1e6, np.inf, -449.0, -1e9, np.nan], dtype=np.float32)
+    got = orc.quantize_e4m3(y)
+    assert got.tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F], got.tolist()
+
+
+def pin_fp8_decode_equals_dequantized_decode(orc):
+    """With power-of-two scales every decoded element is exact in fp16, so
+    the FP8 decode must equal the (pinned) 16-bit decode of those values."""
+    rng = np.random.default_rng(18)
+    lens = [1, 16, 17, 70]
+    H, Hk, D = 4, 2, 32
+    k_scale, v_scale = 2.0 ** -6, 2.0 ** -5
+    p16 = Paged(rng, lens, H, Hk, D, "f16")
+    NB = p16.k_cache.shape[0]
+    kc = rng.integers(0, 0x7f, size=(NB, Hk, 16, D), dtype=np.uint8) | (rng.integers(0, 2, (NB, Hk, 16, D)) << 7).astype(np.uint8)
+    vc = rng.integers(0, 0x7f, size=(NB, Hk, 16, D), dtype=np.uint8) | (rng.integers(0, 2, (NB, Hk, 16, D)) << 7).astype(np.uint8)
+    k16 = narrow(e4m3_torch(kc) * k_scale, "f16")
+    v16 = narrow(e4m3_torch(vc) * v_scale, "f16")
+    assert np.array_equal(widen(k16, "f16"), e4m3_torch(kc) * k_scale), "scaled values must be exact in fp16"
+    want = orc.paged_decode(p16.q, k16, v16, p16.tables, p16.lens, 0.2, "f16")
+    got = orc.paged_decode_fp8(p16.q, kc, vc, p16.tables, p16.lens, 0.2, k_scale, v_scale, "f16")
+    assert np.array_equal(got, want), "FP8 decode differs from the dequantized 16-bit decode"
+
+
+def pin_fp8_cache_write_matches_indexing(orc):
+    rng = np.random.default_rng(19)
+    NB, Hk, B, D = 6, 2, 16, 16
+    kc = rng.integers(0, 255, size=(NB, Hk, B, D), dtype=np.uint8)
+    vc = rng.integers(0, 255, size=(NB, Hk, B, D), dtype=np.uint8)
+    T = 20
+    slots = rng.choice(NB * B, size=T, replace=False).astype(np.int64)
+    slots[4] = -1
+    key = rand_bits(rng, (T, Hk, D), "bf16", -2, 2)
+    val = rand_bits(rng, (T, Hk, D), "bf16", -2, 2)
+    ks, vs = np.float32(1 / 200), np.float32(1 / 150)
+    ek, ev = kc.copy(), vc.copy()
+    live = slots >= 0
+    qk = torch.from_numpy(widen(key, "bf16").astype(np.float32) / ks).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    qv = torch.from_numpy(widen(val, "bf16").astype(np.float32) / vs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ek[slots[live] // B, :, slots[live] % B, :] = qk[live]
+    ev[slots[live] // B, :, slots[live] % B, :] = qv[live]
+    orc.reshape_and_cache_fp8(kc, vc, key, val, slots, "bf16", float(ks), float(vs))
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "FP8 cache write differs"
+
+
 def pin_brute_force_tiny(orc):
     """The first scenario (4 seqs, lengths 1/17/33/100) against the pure
     Python brute force, every (sequence, head)."""

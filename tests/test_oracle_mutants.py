@@ -46,6 +46,14 @@ MUTANTS = {
                       "memmove(k_caches[l] + src * elems, k_caches[l] + dst * elems"),
     "swap_only_k": ("memcpy(dst_v + dst * elems, src_v + src * elems, sizeof(uint16_t) * elems);", ""),
     "swap_direction": ("memcpy(dst_k + dst * elems, src_k + src * elems", "memcpy(dst_k + src * elems, src_k + dst * elems"),
+    "e4m3_exponent_bias": ("v = ldexp((double)(m + 8), e - 10);", "v = ldexp((double)(m + 8), e - 9);"),
+    "e4m3_ties_to_odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "fp8_k_scale_dropped": ("* (widen_e4m3(k_cache[row + d]) * k_scale);", "* widen_e4m3(k_cache[row + d]);"),
+    "fp8_scales_swapped": ("o[d] += w * (widen_e4m3(v_cache[row + d]) * v_scale);",
+                           "o[d] += w * (widen_e4m3(v_cache[row + d]) * k_scale);"),
+    "fp8_write_scale_multiplied": ("quantize_e4m3((float)widen(key[src + d], dtype) / k_scale)",
+                                   "quantize_e4m3((float)widen(key[src + d], dtype) * k_scale)"),
     "zero_length_not_zeroed": ("for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;\n        if (n == 0) continue;",
                                "if (n == 0) { o[0] = 1.0; continue; }\n        "
                                "for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;"),
