@@ -32,9 +32,18 @@ _lib = None
 
 
 def build(src: str = _SRC, out: str = _LIB, extra: Sequence[str] = ()) -> str:
-    """Compile the C oracle with gcc into a shared library and return its path."""
-    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", *extra, "-o", out, src, "-lm"]
-    subprocess.run(cmd, check=True)
+    """Compile the C oracle with gcc into a shared library and return its path.
+
+    The library is written to a temporary name and renamed over ``out``, so a
+    process that already has the old library mapped keeps a valid mapping."""
+    tmp = f"{out}.tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", *extra, "-o", tmp, src, "-lm"]
+    try:
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    finally:
+        if os.path.exists(tmp):
+            os.remove(tmp)
     return out
 
 

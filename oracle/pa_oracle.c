@@ -115,14 +115,26 @@ static double widen_e4m3(uint8_t c) {
     return sign ? -v : v;
 }
 
-/* Nearest E4M3 code to y (ties to the even code), clamped to +-448. */
-static uint8_t quantize_e4m3(float y) {
+/* Magnitudes of the positive finite E4M3 codes 0x01 .. 0x7e, in code order
+ * (which is ascending order of value), widened once per call so that the
+ * nearest-code search below reads a table instead of re-widening. */
+typedef struct {
+    double v[0x7f];
+} e4m3_table;
+
+static void e4m3_table_fill(e4m3_table *t) {
+    for (int c = 0; c < 0x7f; ++c) t->v[c] = widen_e4m3((uint8_t)c);
+}
+
+/* Nearest E4M3 code to y (ties to the even code), clamped to +-448: a
+ * search over every positive finite code. */
+static uint8_t quantize_e4m3(float y, const e4m3_table *t) {
     if (y != y) return 0x7f;
     double a = fabs((double)y);
     uint8_t best = 0;
     double best_err = a;  /* code 0 = +0 */
     for (uint8_t c = 1; c < 0x7f; ++c) {  /* every positive finite code, ascending */
-        double err = fabs(widen_e4m3(c) - a);
+        double err = fabs(t->v[c] - a);
         if (err < best_err || (err == best_err && (c & 1) == 0)) {
             best = c;
             best_err = err;
@@ -133,7 +145,9 @@ static uint8_t quantize_e4m3(float y) {
 }
 
 void oracle_quantize_e4m3_n(uint8_t *out, const float *y, int64_t n) {
-    for (int64_t i = 0; i < n; ++i) out[i] = quantize_e4m3(y[i]);
+    e4m3_table t;
+    e4m3_table_fill(&t);
+    for (int64_t i = 0; i < n; ++i) out[i] = quantize_e4m3(y[i], &t);
 }
 void oracle_widen_e4m3_n(double *out, const uint8_t *c, int64_t n) {
     for (int64_t i = 0; i < n; ++i) out[i] = widen_e4m3(c[i]);
@@ -413,16 +427,21 @@ int oracle_reshape_and_cache_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint1
     if (dtype != ORC_F16 && dtype != ORC_BF16) return ORC_ERR_ARG;
     for (int32_t t = 0; t < num_tokens; ++t)
         if (slot_mapping[t] >= 0 && slot_mapping[t] / block_size >= num_blocks) return ORC_ERR_RANGE;
-    for (int32_t t = 0; t < num_tokens; ++t) {
-        int64_t slot = slot_mapping[t];
-        if (slot < 0) continue;
-        int64_t blk = slot / block_size, off = slot % block_size;
-        for (int32_t h = 0; h < num_kv_heads; ++h) {
+    e4m3_table tab;
+    e4m3_table_fill(&tab);
+    /* heads write disjoint rows, so they may run in parallel; tokens stay in
+     * order within a head */
+#pragma omp parallel for schedule(static)
+    for (int32_t h = 0; h < num_kv_heads; ++h) {
+        for (int32_t t = 0; t < num_tokens; ++t) {
+            int64_t slot = slot_mapping[t];
+            if (slot < 0) continue;
+            int64_t blk = slot / block_size, off = slot % block_size;
             int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
             int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
             for (int32_t d = 0; d < head_dim; ++d) {
-                k_cache[dst + d] = quantize_e4m3((float)widen(key[src + d], dtype) / k_scale);
-                v_cache[dst + d] = quantize_e4m3((float)widen(value[src + d], dtype) / v_scale);
+                k_cache[dst + d] = quantize_e4m3((float)widen(key[src + d], dtype) / k_scale, &tab);
+                v_cache[dst + d] = quantize_e4m3((float)widen(value[src + d], dtype) / v_scale, &tab);
             }
         }
     }

@@ -5,13 +5,33 @@ Each mutant is a copy of ``oracle/pa_oracle.c`` with one textual change
 operand), compiled with gcc into a temporary library and run against the pin
 suite.  A mutant that passes every pin would mean the pins cannot tell that
 mistake from the correct oracle.  Only the CPU oracle is mutated.
+
+The pins run in a child process: a mutant with a wrong index may read or
+write out of bounds, and a crash there must not take the test run with it.
+A crashed child counts as a caught mutant (it did not pass the pins).
 """
 import os
+import subprocess
+import sys
 
 import pytest
 
 import oracle
+
+_CHILD = """
+import sys
+sys.path[:0] = [{tests!r}, {root!r}]
+import oracle
 from pins import ALL_PINS
+orc = oracle.load({lib!r})
+for pin in ALL_PINS:
+    try:
+        pin(orc)
+    except (AssertionError, oracle.OracleError):
+        print("CAUGHT", pin.__name__)
+        sys.exit(0)
+print("PASSED_ALL")
+"""
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
 
@@ -52,8 +72,8 @@ MUTANTS = {
     "fp8_k_scale_dropped": ("* (widen_e4m3(k_cache[row + d]) * k_scale);", "* widen_e4m3(k_cache[row + d]);"),
     "fp8_scales_swapped": ("o[d] += w * (widen_e4m3(v_cache[row + d]) * v_scale);",
                            "o[d] += w * (widen_e4m3(v_cache[row + d]) * k_scale);"),
-    "fp8_write_scale_multiplied": ("quantize_e4m3((float)widen(key[src + d], dtype) / k_scale)",
-                                   "quantize_e4m3((float)widen(key[src + d], dtype) * k_scale)"),
+    "fp8_write_scale_multiplied": ("quantize_e4m3((float)widen(key[src + d], dtype) / k_scale, &tab)",
+                                   "quantize_e4m3((float)widen(key[src + d], dtype) * k_scale, &tab)"),
     "zero_length_not_zeroed": ("for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;\n        if (n == 0) continue;",
                                "if (n == 0) { o[0] = 1.0; continue; }\n        "
                                "for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;"),
@@ -68,12 +88,11 @@ def test_mutant_is_caught(name, tmp_path):
     path = tmp_path / "mutant.c"
     path.write_text(src.replace(old, new))
     lib = oracle.build(str(path), str(tmp_path / "libmutant.so"))
-    orc = oracle.load(lib)
-    failed = []
-    for pin in ALL_PINS:
-        try:
-            pin(orc)
-        except (AssertionError, oracle.OracleError) as e:  # noqa: PERF203
-            failed.append(pin.__name__)
-            break
-    assert failed, f"mutant {name} passed every pin"
+    tests = os.path.dirname(os.path.abspath(__file__))
+    code = _CHILD.format(tests=tests, root=os.path.dirname(tests), lib=lib)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600,
+                       env={**os.environ, "OMP_NUM_THREADS": "2"})
+    if r.returncode < 0:
+        return  # killed by a signal (an out-of-bounds access): caught
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert "PASSED_ALL" not in r.stdout, f"mutant {name} passed every pin"
