@@ -53,13 +53,21 @@ def parse_args(argv=None):
     ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
     ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
+    ap.add_argument("--kv", choices=["16", "fp8"], default="16",
+                    help="KV cache element type: the 16-bit dtype of the workload, or FP8 E4M3 with scales")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     return ap.parse_args(argv)
 
 
-def make_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
+def make_scenario(name: str, seed: int, num_seqs=None, num_blocks=None, kv: str = "16"):
+    from paged_kv_cache_424_b200 import workload as W
+    sc = _base_scenario(name, seed, num_seqs, num_blocks)
+    return W.with_fp8_cache(sc) if kv == "fp8" else sc
+
+
+def _base_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
     from paged_kv_cache_424_b200 import workload as W
     kw = {}
     if num_seqs is not None:
@@ -212,9 +220,7 @@ def cpu_baseline(sc, seconds: float):
         sel = (np.arange(n) + reps * n) % S
         t0 = time.perf_counter()
         for w in st.writes:   # the step's cache write, on the host pool
-            sm = ses.pool.relabel_slots(w.slot_mapping, sc.dims.block_size)
-            k, v = ses.pool.view()
-            orc.reshape_and_cache(k, v, w.key, w.value, sm)
+            ses.write(w.key, w.value, w.slot_mapping)
         ses.decode(st, sel)
         t_total += time.perf_counter() - t0
         seqs_done += n
@@ -243,9 +249,10 @@ def run_ours(args):
     from paged_kv_cache_424_b200 import workload as W
     from paged_kv_cache_424_b200.session import DeviceSession, to_device
 
-    sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks)
+    sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv)
     st = sc.steps[0]
     d = sc.dims
+    fp8 = sc.kv_dtype == "fp8"
     P = sc.partition_tokens if args.partition is None else args.partition
     dev = DeviceSession(sc, device=str(device))
     dev.apply_cache_ops(st)                      # prefill admission + first writes (untimed set-up)
@@ -259,15 +266,29 @@ def run_ours(args):
     out = torch.empty((d.num_seqs, d.num_heads, d.head_dim), dtype=dev.dtype, device=device)
     stream = torch.cuda.current_stream(device)
 
+    def write(key, value, slots):
+        if fp8:
+            pa.pa_reshape_and_cache_fp8(key, value, dev.k_cache, dev.v_cache, slots, sc.k_scale, sc.v_scale,
+                                        stream=stream)
+        else:
+            pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
+
+    def decode(q, bt, cl):
+        if fp8:
+            pa.pa_decode_fp8(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.k_scale, sc.v_scale,
+                             d.num_kv_heads, maxlen, P, ws, stream=stream)
+        else:
+            pa.pa_decode(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, d.num_kv_heads, maxlen, P, ws,
+                         stream=stream)
+
     def step(e0=None, e1=None):
         if bm is not None:
             pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], bm, stream=stream)
         for key, value, slots in writes:
-            pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
+            write(key, value, slots)
         if e0 is not None:
             e0.record(stream)
-        pa.pa_decode(out, inp["q"], dev.k_cache, dev.v_cache, inp["block_tables"], inp["context_lens"], sc.scale,
-                     d.num_kv_heads, maxlen, P, ws, stream=stream)
+        decode(inp["q"], inp["block_tables"], inp["context_lens"])
         if e1 is not None:
             e1.record(stream)
 
@@ -327,9 +348,8 @@ def run_ours(args):
                 d_bm.copy_(h_bm_t, non_blocking=True)
                 pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], d_bm, stream=stream)
             for dk, dv, ds in d_w:
-                pa.pa_reshape_and_cache(dk, dv, dev.k_cache, dev.v_cache, ds, stream=stream)
-            pa.pa_decode(out, d_q, dev.k_cache, dev.v_cache, d_bt, d_cl, sc.scale, d.num_kv_heads, maxlen, P, ws,
-                         stream=stream)
+                write(dk, dv, ds)
+            decode(d_q, d_bt, d_cl)
             h_out.copy_(out, non_blocking=True)
 
         for _ in range(min(args.warmup, 10)):
@@ -355,12 +375,12 @@ def run_ours(args):
 
     # Algorithmic bytes: KV of the referenced tokens; blocks shared by several
     # sequences (copy-on-write prefixes) count once, as the pool holds them once.
-    kv_logical = W.kv_bytes(st, d)
-    kv = W.kv_bytes(st, d, unique=True) if args.workload == "cow" else kv_logical
+    kv_logical = W.kv_bytes(st, d, elem_bytes=sc.kv_elem_bytes)
+    kv = W.kv_bytes(st, d, unique=True, elem_bytes=sc.kv_elem_bytes) if args.workload == "cow" else kv_logical
     algo = kv + W.qo_bytes(d)
     peak, peak_kind = measured_hbm_peak()
     achieved = algo / (dec_avg_ms / 1e3) / 1e9
-    traffic = ncu_traffic(args.workload, units=float(st.context_lens.sum()))
+    traffic = ncu_traffic(args.workload + ("-fp8" if fp8 else ""), units=float(st.context_lens.sum()))
     result = {
         "metric": METRIC,
         "value": d.num_seqs * K * world / (ms_total / 1e3),
@@ -372,7 +392,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": d.dtype,
+        "dtype": f"{d.dtype} q/out, e4m3 KV cache" if fp8 else d.dtype,
         "data": "synthetic (seeded U[-1,1] fp16/bf16 values, NaN in every unused slot; no dataset)",
         "config": {"workload": f"{sc.name}: {sc.note}", "global_batch": d.num_seqs * world,
                    "seq_len": "per-sequence, " + f"mean {float(st.context_lens.mean()):.0f}, "
@@ -384,7 +404,8 @@ def run_ours(args):
                    "algorithmic_bytes_per_step": algo},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": "pa_decode (decode kernel + log-sum-exp merge)" if nparts > 1 else "pa_decode",
+                     "kernel": ("pa_decode_fp8" if fp8 else "pa_decode") +
+                               (" (decode kernel + log-sum-exp merge)" if nparts > 1 else ""),
                      "kernel_ms": dec_avg_ms, "frac_of_8000": achieved / 8000.0,
                      "effective_gbs_logical": (kv_logical + W.qo_bytes(d)) / (dec_avg_ms / 1e3) / 1e9},
         "clocks": clocks.summary(),
@@ -411,7 +432,7 @@ def run_reference(args):
     from oracle.harness import OracleSession
     orc = oracle.load()
     cores = orc.max_threads()
-    sc = make_scenario(args.workload, seed=1, num_seqs=args.num_seqs, num_blocks=args.num_blocks)
+    sc = make_scenario(args.workload, seed=1, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv)
     st = sc.steps[0]
     S = sc.dims.num_seqs
     ses = OracleSession(sc, oracle=orc)
@@ -425,9 +446,7 @@ def run_reference(args):
     def one(i):
         sel = (np.arange(n) + i * n) % S
         for w in st.writes:
-            sm = ses.pool.relabel_slots(w.slot_mapping, sc.dims.block_size)
-            k, v = ses.pool.view()
-            orc.reshape_and_cache(k, v, w.key, w.value, sm)
+            ses.write(w.key, w.value, w.slot_mapping)
         ses.decode(st, sel)
 
     for i in range(args.warmup):

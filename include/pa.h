@@ -7,6 +7,7 @@
  *   pa_reshape_and_cache  write each new token's key/value into its slot
  *   pa_copy_blocks        copy-on-write duplication of shared blocks
  *   pa_swap_blocks        block copies between device and host pools (preemption)
+ *   pa_decode_fp8, pa_reshape_and_cache_fp8   the same over FP8 E4M3 caches
  *   pa_decode             single-query attention of every sequence over its
  *                         cached tokens, gathered through its block table
  *
@@ -69,7 +70,11 @@ typedef enum pa_status {
     PA_ERR_MEMORY = -8       /* a pointer the device cannot address (pageable host memory) */
 } pa_status;
 
-typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+typedef enum pa_dtype {
+    PA_F16 = 0,
+    PA_BF16 = 1,
+    PA_FP8_E4M3 = 2 /* KV caches only: OCP FP8 E4M3 codes, one fp32 scale per tensor */
+} pa_dtype;
 
 /* Bits of the device error word (pa_device_error). */
 #define PA_DEVERR_BLOCK_ID 1u    /* a block-table entry outside [0, num_blocks) */
@@ -88,7 +93,9 @@ typedef struct pa_dims {
     int32_t block_size;         /* B: tokens per block, 16 */
     int32_t max_blocks_per_seq; /* MB: row stride of block_tables */
     int64_t num_blocks;         /* NB: physical blocks in each cache */
-    int32_t dtype;              /* pa_dtype */
+    int32_t dtype;              /* pa_dtype of q, out, key, value (PA_F16 / PA_BF16) */
+    int32_t kv_dtype;           /* pa_dtype of the K / V caches; 0 (= PA_F16) or the value of
+                                   dtype means "same as dtype", PA_FP8_E4M3 an FP8 cache */
 } pa_dims;
 
 /*
@@ -166,6 +173,32 @@ pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const
                             int32_t partition_tokens, void *stream);
 
 /*
+ * Decode attention over FP8 E4M3 caches (dims->kv_dtype == PA_FP8_E4M3), a
+ * variant of pa_decode that reads half the bytes.  The pages name FP8 for
+ * weights ("vLLM PagedAttention 大模型推理架构深度实战" section 5.2) and
+ * KV-cache compression as a goal (section 九 item 3).  Same definition as
+ * pa_decode with K_s[j] = decode(k code) * k_scale and V_s[j] = decode(v code)
+ * * v_scale; q / out in dims->dtype.  Runs on the CUDA-core kernel for every
+ * group size; workspace as from pa_decode_workspace_size with the same dims.
+ */
+pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens, float scale,
+                        float k_scale, float v_scale, int32_t num_kv_heads, const pa_dims *dims,
+                        int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * Cache write into FP8 E4M3 caches: for every token t with slot >= 0 and KV
+ * head h, each element of key[t, h, :] (dims->dtype) becomes the E4M3 code
+ * nearest to float(x) / k_scale (one correctly rounded fp32 division; ties to
+ * the even code; magnitudes beyond 448 clamp to 448; NaN stays NaN); the same
+ * for value with v_scale.  One kernel on `stream`.
+ */
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                   const int64_t *slot_mapping, int32_t num_tokens, const pa_dims *dims,
+                                   float k_scale, float v_scale, void *stream);
+
+/*
  * Cache write (ybb.press section 六, "write into the KV cache block").
  * For every token t < num_tokens with slot = slot_mapping[t] >= 0 and every
  * KV head h:
@@ -199,7 +232,7 @@ pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t n
  * (src, dst) = block_mapping[i]:
  *     dst_k[dst] = src_k[src],   dst_v[dst] = src_v[src]
  * (all num_kv_heads * 16 * head_dim elements of a block; dims gives the block
- * geometry and dtype, dims->num_blocks is not used).  The source pools hold
+ * geometry and dims->kv_dtype the element size, dims->num_blocks is not used).  The source pools hold
  * src_num_blocks blocks, the destination pools dst_num_blocks.  Each pool may
  * be device memory or page-locked host memory the device can address with
  * the same pointer (cudaHostAlloc / cudaHostRegister under unified

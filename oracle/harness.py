@@ -17,22 +17,24 @@ import numpy as np
 
 from . import load
 
-NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0}
+NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0, "fp8": 0x7F}
 
 
 class HostPool:
-    """Compact host mirror of a paged K/V pool (uint16 bit patterns)."""
+    """Compact host mirror of a paged K/V pool: uint16 bit patterns of a
+    16-bit cache, or uint8 codes of an FP8 E4M3 cache (``dtype="fp8"``)."""
 
     def __init__(self, num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
                  dtype: str, capacity: int = 64):
         self.num_blocks = num_blocks
         self.shape = (num_kv_heads, block_size, head_dim)
         self.dtype = dtype
+        self.store = np.uint8 if dtype == "fp8" else np.uint16
         self.row_of = np.full(num_blocks, -1, dtype=np.int64)
         self.ids: List[int] = []
         cap = max(1, capacity)
-        self.k = np.full((cap, *self.shape), NAN_BITS[dtype], dtype=np.uint16)
-        self.v = np.full((cap, *self.shape), NAN_BITS[dtype], dtype=np.uint16)
+        self.k = np.full((cap, *self.shape), NAN_BITS[dtype], dtype=self.store)
+        self.v = np.full((cap, *self.shape), NAN_BITS[dtype], dtype=self.store)
         self.n = 0
 
     def _grow(self, need: int) -> None:
@@ -42,7 +44,7 @@ class HostPool:
         new = max(need, 2 * cap)
         for name in ("k", "v"):
             old = getattr(self, name)
-            arr = np.full((new, *self.shape), NAN_BITS[self.dtype], dtype=np.uint16)
+            arr = np.full((new, *self.shape), NAN_BITS[self.dtype], dtype=self.store)
             arr[:self.n] = old[:self.n]
             setattr(self, name, arr)
 
@@ -95,28 +97,58 @@ class HostPool:
         return self.k[:self.n], self.v[:self.n]
 
 
+def _as_u16(a: np.ndarray) -> np.ndarray:
+    """A uint8 pool seen as uint16 pairs (block copies move bytes, so the
+    16-bit copy routine copies an FP8 block exactly)."""
+    return a if a.dtype == np.uint16 else a.view(np.uint16)
+
+
 class OracleSession:
-    """Applies :class:`Step` objects in order: admit, copy, writes, decode."""
+    """Applies :class:`Step` objects in order: admit, copy, writes, decode.
+
+    Over an FP8 cache (``scenario.kv_dtype == "fp8"``) admitted 16-bit blocks
+    and new tokens enter the pool through the oracle's quantising cache
+    write, and decode reads the codes with the scenario's scales."""
 
     def __init__(self, scenario, oracle=None):
         self.sc = scenario
         d = scenario.dims
+        self.fp8 = getattr(scenario, "kv_dtype", "") == "fp8"
         self.orc = oracle if oracle is not None else load()
-        self.pool = HostPool(d.num_blocks, d.num_kv_heads, d.block_size, d.head_dim, d.dtype)
+        self.pool = HostPool(d.num_blocks, d.num_kv_heads, d.block_size, d.head_dim,
+                             "fp8" if self.fp8 else d.dtype)
+
+    def write(self, key, value, slot_mapping) -> None:
+        """The cache write of tokens (16-bit bit patterns) into their slots."""
+        d = self.sc.dims
+        sm = self.pool.relabel_slots(slot_mapping, d.block_size)
+        k, v = self.pool.view()
+        if self.fp8:
+            self.orc.reshape_and_cache_fp8(k, v, key, value, sm, d.dtype, self.sc.k_scale, self.sc.v_scale)
+        else:
+            self.orc.reshape_and_cache(k, v, key, value, sm)
 
     def apply_cache_ops(self, step) -> None:
         d = self.sc.dims
         if step.admit_ids.size:
-            self.pool.admit(step.admit_ids, step.admit_k, step.admit_v)
+            if self.fp8:
+                # every slot of each admitted block, token-major, through the cache write
+                ids = np.asarray(step.admit_ids, np.int64)
+                B = d.block_size
+                self.pool.rows(ids)
+                key = np.ascontiguousarray(step.admit_k.transpose(0, 2, 1, 3)).reshape(-1, d.num_kv_heads, d.head_dim)
+                val = np.ascontiguousarray(step.admit_v.transpose(0, 2, 1, 3)).reshape(-1, d.num_kv_heads, d.head_dim)
+                slots = (ids[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+                self.write(key, val, slots)
+            else:
+                self.pool.admit(step.admit_ids, step.admit_k, step.admit_v)
         if step.block_mapping.size:
             bm = step.block_mapping.reshape(-1, 2)
             rel = np.stack([self.pool.rows(bm[:, 0]), self.pool.rows(bm[:, 1])], axis=1)
             k, v = self.pool.view()
-            self.orc.copy_blocks([k], [v], rel)
+            self.orc.copy_blocks([_as_u16(k)], [_as_u16(v)], rel)
         for w in step.writes:
-            sm = self.pool.relabel_slots(w.slot_mapping, d.block_size)
-            k, v = self.pool.view()
-            self.orc.reshape_and_cache(k, v, w.key, w.value, sm)
+            self.write(w.key, w.value, w.slot_mapping)
 
     def decode(self, step, seqs: Optional[np.ndarray] = None) -> np.ndarray:
         """float64 ``[S, H, D]`` (or only the rows ``seqs``)."""
@@ -127,6 +159,9 @@ class OracleSession:
             q, bt, cl = q[seqs], bt[seqs], cl[seqs]
         rel = self.pool.relabel_tables(bt, cl, d.block_size)
         k, v = self.pool.view()
+        if self.fp8:
+            return self.orc.paged_decode_fp8(q, k, v, rel, cl, self.sc.scale, self.sc.k_scale, self.sc.v_scale,
+                                             d.dtype)
         return self.orc.paged_decode(q, k, v, rel, cl, self.sc.scale, d.dtype)
 
     def run_step(self, step, seqs: Optional[np.ndarray] = None) -> np.ndarray:

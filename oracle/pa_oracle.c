@@ -127,7 +127,8 @@ static void e4m3_table_fill(e4m3_table *t) {
 }
 
 /* Nearest E4M3 code to y (ties to the even code), clamped to +-448: a
- * search over every positive finite code. */
+ * search over every positive finite code for |y|, then y's sign (so -0.0
+ * and negatives that round to zero give -0, code 0x80). */
 static uint8_t quantize_e4m3(float y, const e4m3_table *t) {
     if (y != y) return 0x7f;
     double a = fabs((double)y);
@@ -141,7 +142,7 @@ static uint8_t quantize_e4m3(float y, const e4m3_table *t) {
         }
     }
     if (a > 448.0) best = 0x7e;  /* saturate to finite */
-    return (uint8_t)(best | (y < 0 ? 0x80 : 0));
+    return (uint8_t)(best | (signbit(y) ? 0x80 : 0));  /* the sign is kept, -0 included */
 }
 
 void oracle_quantize_e4m3_n(uint8_t *out, const float *y, int64_t n) {

@@ -21,13 +21,15 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 PA_OK = 0
 STATUS = {0: "PA_OK", -1: "PA_ERR_NULL", -2: "PA_ERR_DTYPE", -3: "PA_ERR_SHAPE", -4: "PA_ERR_UNSUPPORTED",
           -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_CUDA", -7: "PA_ERR_ALIGN", -8: "PA_ERR_MEMORY"}
-PA_F16, PA_BF16 = 0, 1
-DEVERR = {1: "BLOCK_ID", 2: "CONTEXT", 4: "SLOT", 8: "COPY_PAIR", 16: "TIMEOUT"}
+PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+DEVERR = {1: "BLOCK_ID", 2: "CONTEXT", 4: "SLOT", 8: "COPY_PAIR", 16: "TIMEOUT", 32: "LAYOUT"}
+# torch dtypes accepted for an FP8 E4M3 cache (the codes as bytes, or torch's own e4m3fn type)
+FP8_CACHE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
 # The C entry points declared in include/pa.h, in declaration order.
 EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_decode_noalloc",
-           "pa_reshape_and_cache",
-           "pa_copy_blocks", "pa_swap_blocks", "pa_last_error", "pa_device_error", "pa_version"]
+           "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks",
+           "pa_last_error", "pa_device_error", "pa_version"]
 
 
 class LibraryMissing(RuntimeError):
@@ -43,7 +45,7 @@ class PagedAttentionError(RuntimeError):
 class pa_dims(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
-                ("num_blocks", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+                ("num_blocks", ctypes.c_int64), ("dtype", ctypes.c_int32), ("kv_dtype", ctypes.c_int32)]
 
 
 def _load(path: str = LIB_PATH):
@@ -60,6 +62,11 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, dp, i32, i32, vp]
     lib.pa_decode_noalloc.restype = ctypes.c_int
+    f32 = ctypes.c_float
+    lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, f32, f32, f32, i32, dp, i32, i32, vp, u64, vp]
+    lib.pa_decode_fp8.restype = ctypes.c_int
+    lib.pa_reshape_and_cache_fp8.argtypes = [vp, vp, vp, vp, vp, i32, dp, f32, f32, vp]
+    lib.pa_reshape_and_cache_fp8.restype = ctypes.c_int
     lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, dp, vp]
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
@@ -112,9 +119,14 @@ def _need_cuda(*ts: Optional[torch.Tensor]) -> None:
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _kv_code(cache: torch.Tensor) -> int:
+    return PA_FP8_E4M3 if cache.dtype in FP8_CACHE_DTYPES else _dtype_code(cache)
+
+
 def make_dims(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
-              max_blocks_per_seq: int, num_blocks: int, dtype: int) -> pa_dims:
-    return pa_dims(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype)
+              max_blocks_per_seq: int, num_blocks: int, dtype: int, kv_dtype: int = 0) -> pa_dims:
+    return pa_dims(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype,
+                   kv_dtype)
 
 
 def dims_of(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) -> pa_dims:
@@ -123,12 +135,19 @@ def dims_of(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) 
     if D2 != D:
         raise ValueError("q and k_cache disagree on head_dim")
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
-    return make_dims(S, H, Hk, D, B, MB, NB, _dtype_code(q))
+    return make_dims(S, H, Hk, D, B, MB, NB, _dtype_code(q), _kv_code(k_cache))
 
 
-def cache_dims(k_cache: torch.Tensor) -> pa_dims:
+def cache_dims(k_cache: torch.Tensor, dtype: Optional[torch.dtype] = None) -> pa_dims:
+    """Block geometry of a cache; `dtype` is the 16-bit type of the tokens
+    written into it (taken from the cache itself unless it is FP8)."""
     NB, Hk, B, D = k_cache.shape
-    return make_dims(0, Hk, Hk, D, B, 0, NB, _dtype_code(k_cache))
+    kv = _kv_code(k_cache)
+    if dtype is not None:
+        code = _dtype_code(torch.empty(0, dtype=dtype))
+    else:
+        code = PA_F16 if kv == PA_FP8_E4M3 else kv
+    return make_dims(0, Hk, Hk, D, B, 0, NB, code, kv)
 
 
 # ---------------------------------------------------------------------------
@@ -188,6 +207,41 @@ def pa_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                                int(max_context_len), int(partition_tokens), _stream(stream))
     _check(st)
     return out
+
+
+def pa_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, k_scale: float,
+                  v_scale: float, num_kv_heads: int, max_context_len: int, partition_tokens: int = 0,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pa_decode over FP8 E4M3 caches (uint8 or float8_e4m3fn tensors):
+    K = code * k_scale, V = code * v_scale."""
+    _need_cuda(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if k_cache.dtype not in FP8_CACHE_DTYPES or v_cache.dtype not in FP8_CACHE_DTYPES:
+        raise TypeError("FP8 caches must be uint8 or float8_e4m3fn tensors")
+    dims = dims_of(q, k_cache, block_tables)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = LIB.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                           float(scale), float(k_scale), float(v_scale), int(num_kv_heads), ctypes.byref(dims),
+                           int(max_context_len), int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st)
+    return out
+
+
+def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             slot_mapping: torch.Tensor, k_scale: float, v_scale: float, stream=None) -> None:
+    """k_cache[slot // 16, :, slot % 16] = e4m3(key[t] / k_scale) (and V) for slot >= 0."""
+    _need_cuda(key, value, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if k_cache.dtype not in FP8_CACHE_DTYPES or v_cache.dtype not in FP8_CACHE_DTYPES:
+        raise TypeError("FP8 caches must be uint8 or float8_e4m3fn tensors")
+    dims = cache_dims(k_cache, key.dtype)
+    st = LIB.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                      int(slot_mapping.numel()), ctypes.byref(dims), float(k_scale), float(v_scale),
+                                      _stream(stream))
+    _check(st)
 
 
 def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

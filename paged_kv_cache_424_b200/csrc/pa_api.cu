@@ -2,6 +2,7 @@
 // argument validation, the split-KV plan, and dispatch to the launchers.
 #include <cstdarg>
 #include <cstdint>
+#include <cmath>
 #include <cstdio>
 
 #include "../../include/pa.h"
@@ -35,10 +36,15 @@ constexpr int kAutoPartitionSimt = 512;
 constexpr int kAutoPartitionTc = 1024;
 constexpr int kMaxPartitionTokens = 32768;
 
+bool kv_fp8(const pa_dims *d) { return d->kv_dtype == PA_FP8_E4M3; }
+int32_t kv_elem_bytes(const pa_dims *d) { return kv_fp8(d) ? 1 : 2; }
+
 // Checks of the fields every call uses.  `attention` adds the query-side ones.
 pa_status check_dims(const pa_dims *d, bool attention) {
     if (!d) return fail(PA_ERR_NULL, "dims is NULL");
     if (d->dtype != PA_F16 && d->dtype != PA_BF16) return fail(PA_ERR_DTYPE, "dtype %d is not PA_F16/PA_BF16", d->dtype);
+    if (d->kv_dtype != 0 && d->kv_dtype != d->dtype && d->kv_dtype != PA_FP8_E4M3)
+        return fail(PA_ERR_DTYPE, "kv_dtype %d: must be 0, dtype (%d) or PA_FP8_E4M3", d->kv_dtype, d->dtype);
     if (d->num_kv_heads <= 0 || d->head_dim <= 0 || d->block_size <= 0 || d->num_blocks <= 0)
         return fail(PA_ERR_SHAPE, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
     if (d->block_size != 16) return fail(PA_ERR_UNSUPPORTED, "block_size %d: only 16 is built", d->block_size);
@@ -76,7 +82,7 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
                     partition_tokens, kMaxPartitionTokens);
     const int g = d->num_heads / d->num_kv_heads;
-    const bool tc = pa::decode_tc_supported(d->head_dim, g, d->num_blocks, d->num_kv_heads);
+    const bool tc = !kv_fp8(d) && pa::decode_tc_supported(d->head_dim, g, d->num_blocks, d->num_kv_heads);
     const int P = partition_tokens != 0 ? partition_tokens : tc ? kAutoPartitionTc : kAutoPartitionSimt;
     const int ctx_blocks = (max_context_len + 15) / 16;
     int part_blocks = P / 16;
@@ -90,6 +96,57 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         pl->lse_off = pl->o_bytes;
         pl->ws_bytes = pl->o_bytes + align_up(rows * sizeof(float), 256);
     }
+    return PA_OK;
+}
+
+// Shared body of pa_decode and pa_decode_fp8 (dims already checked).  For a
+// 16-bit cache k_scale = v_scale = 1.
+pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *context_lens, float scale, float k_scale,
+                      float v_scale, int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
+                      int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream) {
+    pa_status st;
+    if (num_kv_heads != dims->num_kv_heads)
+        return fail(PA_ERR_SHAPE, "num_kv_heads %d != dims->num_kv_heads %d", num_kv_heads, dims->num_kv_heads);
+    Plan pl;
+    st = make_plan(dims, max_context_len, partition_tokens, &pl);
+    if (st != PA_OK) return st;
+    if (dims->num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !context_lens || (!block_tables && dims->max_blocks_per_seq > 0))
+        return fail(PA_ERR_NULL, "a required pointer is NULL");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "out, q, k_cache and v_cache must be 16-byte aligned");
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes)
+            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.ws_bytes,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned16(workspace)) return fail(PA_ERR_ALIGN, "workspace must be 16-byte aligned");
+    }
+    pa::DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.scale_log2 = scale * 1.4426950408889634f * k_scale;
+    p.v_scale = v_scale;
+    p.num_seqs = dims->num_seqs;
+    p.num_heads = dims->num_heads;
+    p.num_kv_heads = dims->num_kv_heads;
+    p.max_blocks_per_seq = dims->max_blocks_per_seq;
+    p.num_blocks = dims->num_blocks;
+    p.part_blocks = pl.part_blocks;
+    p.max_parts = pl.max_parts;
+    p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
+    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.lse_off) : nullptr;
+    const int g = dims->num_heads / dims->num_kv_heads;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool fp8 = kv_fp8(dims);
+    cudaError_t e = !fp8 && pa::decode_tc_supported(dims->head_dim, g, dims->num_blocks, dims->num_kv_heads)
+                        ? pa::launch_decode_tc(p, dims->dtype, g, cs)
+                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, g, fp8, cs);
+    if (e != cudaSuccess) return cuda_fail(e, fp8 ? "pa_decode_fp8 launch" : "pa_decode launch");
     return PA_OK;
 }
 
@@ -128,46 +185,22 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     void *stream) {
     pa_status st = check_dims(dims, true);
     if (st != PA_OK) return st;
-    if (num_kv_heads != dims->num_kv_heads)
-        return fail(PA_ERR_SHAPE, "num_kv_heads %d != dims->num_kv_heads %d", num_kv_heads, dims->num_kv_heads);
-    Plan pl;
-    st = make_plan(dims, max_context_len, partition_tokens, &pl);
+    if (kv_fp8(dims)) return fail(PA_ERR_DTYPE, "pa_decode: kv_dtype is PA_FP8_E4M3, call pa_decode_fp8");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, 1.f, 1.f, num_kv_heads, dims,
+                       max_context_len, partition_tokens, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens, float scale, float k_scale,
+                        float v_scale, int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
+                        int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream) {
+    pa_status st = check_dims(dims, true);
     if (st != PA_OK) return st;
-    if (dims->num_seqs == 0) return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !context_lens || (!block_tables && dims->max_blocks_per_seq > 0))
-        return fail(PA_ERR_NULL, "a required pointer is NULL");
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-        return fail(PA_ERR_ALIGN, "out, q, k_cache and v_cache must be 16-byte aligned");
-    if (pl.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < pl.ws_bytes)
-            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.ws_bytes,
-                        workspace ? workspace_bytes : (size_t)0);
-        if (!aligned16(workspace)) return fail(PA_ERR_ALIGN, "workspace must be 16-byte aligned");
-    }
-    pa::DecodeParams p{};
-    p.out = out;
-    p.q = q;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.num_seqs = dims->num_seqs;
-    p.num_heads = dims->num_heads;
-    p.num_kv_heads = dims->num_kv_heads;
-    p.max_blocks_per_seq = dims->max_blocks_per_seq;
-    p.num_blocks = dims->num_blocks;
-    p.part_blocks = pl.part_blocks;
-    p.max_parts = pl.max_parts;
-    p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
-    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.lse_off) : nullptr;
-    const int g = dims->num_heads / dims->num_kv_heads;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    cudaError_t e = pa::decode_tc_supported(dims->head_dim, g, dims->num_blocks, dims->num_kv_heads)
-                        ? pa::launch_decode_tc(p, dims->dtype, g, cs)
-                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, g, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    return PA_OK;
+    if (!kv_fp8(dims)) return fail(PA_ERR_DTYPE, "pa_decode_fp8: dims->kv_dtype must be PA_FP8_E4M3");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
+        return fail(PA_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale, num_kv_heads,
+                       dims, max_context_len, partition_tokens, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
@@ -179,10 +212,31 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
     if (!key || !value || !k_cache || !v_cache || !slot_mapping) return fail(PA_ERR_NULL, "a required pointer is NULL");
     if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
         return fail(PA_ERR_ALIGN, "key, value and caches must be 16-byte aligned");
-    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    if (kv_fp8(dims)) return fail(PA_ERR_DTYPE, "pa_reshape_and_cache: kv_dtype is PA_FP8_E4M3, call pa_reshape_and_cache_fp8");
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks, 2};
     cudaError_t e = pa::launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens, cd,
                                                  static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache launch");
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                   const int64_t *slot_mapping, int32_t num_tokens, const pa_dims *dims,
+                                   float k_scale, float v_scale, void *stream) {
+    pa_status st = check_dims(dims, false);
+    if (st != PA_OK) return st;
+    if (!kv_fp8(dims)) return fail(PA_ERR_DTYPE, "pa_reshape_and_cache_fp8: dims->kv_dtype must be PA_FP8_E4M3");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
+        return fail(PA_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+    if (num_tokens < 0) return fail(PA_ERR_SHAPE, "num_tokens %d < 0", num_tokens);
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return fail(PA_ERR_NULL, "a required pointer is NULL");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "key, value and caches must be 16-byte aligned");
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks, 1};
+    cudaError_t e = pa::launch_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, num_tokens, cd,
+                                                     dims->dtype, k_scale, v_scale, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache_fp8 launch");
     return PA_OK;
 }
 
@@ -199,7 +253,7 @@ pa_status pa_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t n
             return fail(PA_ERR_ALIGN, "cache pointers of layer %d must be 16-byte aligned", i);
     }
     if (num_pairs > 65535) return fail(PA_ERR_SHAPE, "num_pairs %d > 65535", num_pairs);
-    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks, kv_elem_bytes(dims)};
     cudaError_t e = pa::launch_copy_blocks(k_caches, v_caches, num_layers, block_mapping, num_pairs, cd,
                                            static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "pa_copy_blocks launch");
@@ -237,7 +291,7 @@ pa_status pa_swap_blocks(const void *src_k, const void *src_v, int64_t src_num_b
     const void *bm = device_address(block_mapping);
     if (!sk || !sv || !dk || !dv || !bm)
         return fail(PA_ERR_MEMORY, "a pool or the mapping is not device or page-locked host memory");
-    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks};
+    pa::CacheDims cd{dims->num_kv_heads, dims->head_dim, dims->num_blocks, kv_elem_bytes(dims)};
     cudaError_t e = pa::launch_swap_blocks(sk, sv, src_num_blocks, const_cast<void *>(dk), const_cast<void *>(dv),
                                            dst_num_blocks, static_cast<const int64_t *>(bm), num_pairs, cd,
                                            static_cast<cudaStream_t>(stream));

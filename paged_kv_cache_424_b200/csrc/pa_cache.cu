@@ -114,13 +114,76 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// One thread per 16 elements of a (token, kv head) row: two 16-byte loads of
+// key (value), a correctly rounded fp32 division by the tensor's scale, then
+// round-to-nearest-even to E4M3 with saturation, one 16-byte store.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_fp8_kernel(const T *__restrict__ key, const T *__restrict__ value, uint8_t *__restrict__ k_cache,
+                                 uint8_t *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping,
+                                 int64_t num_items, int items_per_row, int head_dim, int num_kv_heads,
+                                 int64_t num_slots, float k_scale, float v_scale) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= num_items) return;
+    const int64_t row = i / items_per_row;  // (token, kv head)
+    const int c = (int)(i % items_per_row);
+    const int64_t t = row / num_kv_heads;
+    const int h = (int)(row % num_kv_heads);
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (h == 0 && c == 0) flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const int64_t blk = slot / kBlock, off = slot % kBlock;
+    const int64_t dst = ((blk * num_kv_heads + h) * kBlock + off) * head_dim + c * 16;
+    auto quantize16 = [&](const T *src, float sc, uint8_t *out) {
+        const uint4 a = reinterpret_cast<const uint4 *>(src)[0];
+        const uint4 b = reinterpret_cast<const uint4 *>(src)[1];
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t packed[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 x0 = Elem<T>::to_float2(w[2 * j]);
+            const float2 x1 = Elem<T>::to_float2(w[2 * j + 1]);
+            const uint16_t lo = float2_to_e4m3x2(__fdiv_rn(x0.x, sc), __fdiv_rn(x0.y, sc));
+            const uint16_t hi = float2_to_e4m3x2(__fdiv_rn(x1.x, sc), __fdiv_rn(x1.y, sc));
+            packed[j] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+        *reinterpret_cast<uint4 *>(out) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    };
+    const int64_t src = row * head_dim + c * 16;
+    quantize16(key + src, k_scale, k_cache + dst);
+    quantize16(value + src, v_scale, v_cache + dst);
+}
+
 }  // namespace
+
+cudaError_t launch_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                         const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,
+                                         int dtype, float k_scale, float v_scale, cudaStream_t stream) {
+    const int ipr = d.head_dim / 16;
+    const int64_t items = (int64_t)num_tokens * d.num_kv_heads * ipr;
+    if (items == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((items + 255) / 256));
+    const int64_t slots = (int64_t)d.num_blocks * kBlock;
+    uint8_t *kc = static_cast<uint8_t *>(k_cache), *vc = static_cast<uint8_t *>(v_cache);
+    if (dtype == PA_F16)
+        return launch_pdl(reshape_and_cache_fp8_kernel<__half>, grid, dim3(256), 0, stream,
+                          static_cast<const __half *>(key), static_cast<const __half *>(value), kc, vc, slot_mapping,
+                          items, ipr, (int)d.head_dim, (int)d.num_kv_heads, slots, k_scale, v_scale);
+    return launch_pdl(reshape_and_cache_fp8_kernel<__nv_bfloat16>, grid, dim3(256), 0, stream,
+                      static_cast<const __nv_bfloat16 *>(key), static_cast<const __nv_bfloat16 *>(value), kc, vc,
+                      slot_mapping, items, ipr, (int)d.head_dim, (int)d.num_kv_heads, slots, k_scale, v_scale);
+}
 
 cudaError_t launch_swap_blocks(const void *src_k, const void *src_v, int64_t src_blocks, void *dst_k, void *dst_v,
                                int64_t dst_blocks, const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
                                cudaStream_t stream) {
     if (num_pairs == 0) return cudaSuccess;
-    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim / 8;
+    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim * d.elem_bytes / 16;
     return launch_pdl(swap_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream, static_cast<const uint4 *>(src_k),
                       static_cast<const uint4 *>(src_v), src_blocks, static_cast<uint4 *>(dst_k),
                       static_cast<uint4 *>(dst_v), dst_blocks, block_mapping, chunks);
@@ -143,7 +206,7 @@ cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int
                                const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
                                cudaStream_t stream) {
     if (num_pairs == 0 || num_layers == 0) return cudaSuccess;
-    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim / 8;
+    const int64_t chunks = (int64_t)d.num_kv_heads * kBlock * d.head_dim * d.elem_bytes / 16;
     for (int l0 = 0; l0 < num_layers; l0 += kCopyLayers) {
         const int nl = num_layers - l0 < kCopyLayers ? num_layers - l0 : kCopyLayers;
         LayerPtrs ptrs = {};

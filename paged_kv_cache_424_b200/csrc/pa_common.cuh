@@ -5,6 +5,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,6 +46,23 @@ template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
     static __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 };
+
+// FP8 E4M3 cache element (stored as its 8-bit code).
+struct E4M3 {
+    uint8_t code;
+};
+
+// Two E4M3 codes (element 0 in the low byte) -> two floats, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t pair) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+
+// Two floats -> two E4M3 codes, nearest with ties to even, clamped to the
+// largest finite magnitude (element 0 in the low byte).
+__device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
+    return __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
 
 // ---------------------------------------------------------------------------
 // shared-memory addresses, mbarriers and bulk copies (PTX ISA: mbarrier,

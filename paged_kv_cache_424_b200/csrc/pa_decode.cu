@@ -46,22 +46,24 @@ __device__ __forceinline__ int part_lmax(const DecodeParams &p) {
 //   [table] part_blocks int32
 struct PartLayout {
     int chunk, main, q_off, p_off, ml_off, bar_off, table_off;
-    __host__ __device__ constexpr PartLayout(int D, int G, int nstage)
-        : chunk(kBlock * D * 2),
-          main(kWarps * nstage * 2 * kBlock * D * 2 > kWarps * G * D * 4 ? kWarps * nstage * 2 * kBlock * D * 2
-                                                                        : kWarps * G * D * 4),
+    __host__ __device__ constexpr PartLayout(int D, int G, int nstage, int esz)
+        : chunk(kBlock * D * esz),
+          main(kWarps * nstage * 2 * kBlock * D * esz > kWarps * G * D * 4 ? kWarps * nstage * 2 * kBlock * D * esz
+                                                                          : kWarps * G * D * 4),
           q_off(main), p_off(q_off + G * 2 * (D / 16) * 12 * 4), ml_off(p_off + kWarps * G * kBlock * 4),
           bar_off((ml_off + 2 * kWarps * G * 4 + 7) / 8 * 8), table_off(bar_off + kWarps * nstage * 8) {}
     __host__ __device__ constexpr int bytes(int part_blocks) const { return table_off + part_blocks * 4; }
 };
 
-// Stages per warp ring: 2 for small groups (3 CTAs / SM, more warps to hide
-// the per-block latency chains), 3 otherwise.
-__host__ __device__ constexpr int part_stages(int G) { return G <= 2 ? 2 : 3; }
+// Stages per warp ring: for 16-bit caches 2 with small groups (3 CTAs / SM,
+// more warps to hide the per-block latency chains), 3 otherwise; FP8 blocks
+// are half the bytes, so twice the stages keep as many bytes in flight.
+__host__ __device__ constexpr int part_stages(int G, int esz) { return (G <= 2 ? 2 : 3) * (esz == 1 ? 2 : 1); }
 
-template <typename T, int D, int G, int NSTAGE>
+template <typename T, typename KT, int D, int G, int NSTAGE>
 __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodeParams p) {
-    constexpr PartLayout S(D, G, NSTAGE);
+    constexpr int kEsz = std::is_same<KT, E4M3>::value ? 1 : 2;
+    constexpr PartLayout S(D, G, NSTAGE, kEsz);
     using E = Elem<T>;
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -110,13 +112,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     unsigned char *stages = smem + warp * NSTAGE * 2 * S.chunk;
     uint64_t *wbar = bars + warp * NSTAGE;
     const int nw = (b1 - b0 - warp + kWarps - 1) / kWarps;  // blocks of this warp (may be <= 0)
-    const T *kc = reinterpret_cast<const T *>(p.k_cache);
-    const T *vc = reinterpret_cast<const T *>(p.v_cache);
+    const unsigned char *kc = reinterpret_cast<const unsigned char *>(p.k_cache);
+    const unsigned char *vc = reinterpret_cast<const unsigned char *>(p.v_cache);
 
     auto issue = [&](int j) {
         const int st = j % NSTAGE;
         const int64_t phys = tbl[warp + kWarps * j];
-        const int64_t off = ((phys * p.num_kv_heads + kvh) * kBlock) * D;
+        const int64_t off = ((phys * p.num_kv_heads + kvh) * kBlock) * D * kEsz;
         unsigned char *dst = stages + st * 2 * S.chunk;
         mbar_arrive_expect_tx(&wbar[st], 2 * S.chunk);
         bulk_g2s(dst, kc + off, S.chunk, &wbar[st]);
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
         }
         const unsigned char *ks = stages + st * 2 * S.chunk;
         const int base = (b0 + warp + kWarps * j) * kBlock;
-        simt_block<T, D, G>(state, ks, ks + S.chunk, min(kBlock, L - base), q_s, pw, lane);
+        simt_block<T, KT, D, G>(state, ks, ks + S.chunk, min(kBlock, L - base), q_s, pw, lane);
         if (lane == 0 && j + NSTAGE < nw) {
             fence_proxy_async_smem();
             issue(j + NSTAGE);
@@ -169,7 +171,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     for (int i = tid; i < G * D; i += blockDim.x) {
         const int h = i / D, d = i % D;
         float lse;
-        const float o = combine_warps<D, G, kWarps>(red_m, red_l, red_acc, h, d, &lse);
+        float o = combine_warps<D, G, kWarps>(red_m, red_l, red_acc, h, d, &lse);
+        if constexpr (kEsz == 1) o *= p.v_scale;  // FP8: V codes were unscaled
         const int head = head0 + h;
         if (direct) {
             out[((int64_t)s * H + head) * D + d] = E::from_float(o);
@@ -205,10 +208,12 @@ __global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p) {
     reinterpret_cast<T *>(p.out)[((int64_t)s * p.num_heads + h) * D + d] = Elem<T>::from_float(o / wsum);
 }
 
-template <typename T, int D, int G>
+template <typename T, typename KT, int D, int G>
 cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
-    auto kern = decode_part_kernel<T, D, G, part_stages(G)>;
-    const int smem = PartLayout(D, G, part_stages(G)).bytes(p.part_blocks);
+    constexpr int kEsz = std::is_same<KT, E4M3>::value ? 1 : 2;
+    constexpr int kStages = part_stages(G, kEsz);
+    auto kern = decode_part_kernel<T, KT, D, G, kStages>;
+    const int smem = PartLayout(D, G, kStages, kEsz).bytes(p.part_blocks);
     static int configured[kMaxDevices] = {};
     cudaError_t e = ensure_smem(kern, smem, configured);
     if (e != cudaSuccess) return e;
@@ -217,16 +222,21 @@ cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, D, stream);
 }
 
-template <typename T, int D>
+template <typename T, typename KT, int D>
 cudaError_t launch_part_d(const DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_part_t<T, D, 1>(p, stream);
-        case 2: return launch_part_t<T, D, 2>(p, stream);
-        case 4: return launch_part_t<T, D, 4>(p, stream);
-        case 8: return launch_part_t<T, D, 8>(p, stream);
-        case 16: return launch_part_t<T, D, 16>(p, stream);
+        case 1: return launch_part_t<T, KT, D, 1>(p, stream);
+        case 2: return launch_part_t<T, KT, D, 2>(p, stream);
+        case 4: return launch_part_t<T, KT, D, 4>(p, stream);
+        case 8: return launch_part_t<T, KT, D, 8>(p, stream);
+        case 16: return launch_part_t<T, KT, D, 16>(p, stream);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <typename T, typename KT>
+cudaError_t launch_part_k(const DecodeParams &p, int head_dim, int group, cudaStream_t stream) {
+    return head_dim == 64 ? launch_part_d<T, KT, 64>(p, group, stream) : launch_part_d<T, KT, 128>(p, group, stream);
 }
 
 }  // namespace
@@ -240,13 +250,13 @@ cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_d
                           : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p);
 }
 
-cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group,
+cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group, bool fp8_cache,
                                       cudaStream_t stream) {
     if (dtype == PA_F16)
-        return head_dim == 64 ? launch_part_d<__half, 64>(p, group, stream)
-                              : launch_part_d<__half, 128>(p, group, stream);
-    return head_dim == 64 ? launch_part_d<__nv_bfloat16, 64>(p, group, stream)
-                          : launch_part_d<__nv_bfloat16, 128>(p, group, stream);
+        return fp8_cache ? launch_part_k<__half, E4M3>(p, head_dim, group, stream)
+                         : launch_part_k<__half, __half>(p, head_dim, group, stream);
+    return fp8_cache ? launch_part_k<__nv_bfloat16, E4M3>(p, head_dim, group, stream)
+                     : launch_part_k<__nv_bfloat16, __nv_bfloat16>(p, head_dim, group, stream);
 }
 
 }  // namespace pa

@@ -21,7 +21,8 @@ struct DecodeParams {
     const int32_t *context_lens; // [S]
     float *ws_o;                 // [S, H, max_parts, D] partial outputs (split only)
     float *ws_lse;               // [S, H, max_parts] log2-sum-exp per partial
-    float scale_log2;            // scale * log2(e)
+    float scale_log2;            // scale * log2(e) (times k_scale for an FP8 cache)
+    float v_scale;               // applied to the output (1 unless the cache is FP8)
     int32_t num_seqs, num_heads, num_kv_heads, max_blocks_per_seq;
     int64_t num_blocks;
     int32_t part_blocks;         // table entries per KV partition
@@ -47,8 +48,9 @@ inline cudaError_t ensure_smem(K kern, int bytes, int *configured_per_device) {
 // Record `msg` as the text pa_last_error() returns on this thread; returns st.
 pa_status set_last_error(pa_status st, const char *msg);
 
-// Fixed-partition decode (+ merge when max_parts > 1) on `stream`.
-cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group,
+// Fixed-partition decode (+ merge when max_parts > 1) on `stream`; the
+// caches hold elements of `dtype`, or FP8 E4M3 codes when `fp8_cache`.
+cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group, bool fp8_cache,
                                       cudaStream_t stream);
 
 
@@ -64,10 +66,14 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int group, cudaSt
 struct CacheDims {
     int32_t num_kv_heads, head_dim;
     int64_t num_blocks;
+    int32_t elem_bytes;  // 2 for fp16 / bf16, 1 for FP8 E4M3
 };
 cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
                                      const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,
                                      cudaStream_t stream);
+cudaError_t launch_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                         const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,
+                                         int dtype, float k_scale, float v_scale, cudaStream_t stream);
 cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
                                const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
                                cudaStream_t stream);

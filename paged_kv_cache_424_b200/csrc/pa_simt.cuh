@@ -16,6 +16,8 @@
 // others are masked to weight 0 and their V rows are never read.
 #pragma once
 
+#include <type_traits>
+
 #include "pa_common.cuh"
 #include "pa_decode.h"
 
@@ -105,11 +107,15 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // One warp folds one block into `st`.  ks / vs: the K and V chunks in shared
-// memory; pw: this warp's G x 16 float scratch for the softmax weights.
-template <typename T, int D, int G>
+// memory, elements of KT (T itself, or E4M3 codes whose scale the caller
+// folds into q and the output); pw: this warp's G x 16 float scratch for the
+// softmax weights.
+template <typename T, typename KT, int D, int G>
 __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned char *ks, const unsigned char *vs,
                                            int nvalid, const float *q_s, float *pw, int lane) {
     using E = Elem<T>;
+    constexpr bool kFp8 = std::is_same<KT, E4M3>::value;
+    constexpr int kEsz = kFp8 ? 1 : 2;   // bytes per cache element
     constexpr int kNC = SimtQ<D>::kNC;
     constexpr int kPV = SimtState<D, G>::kPV;
     constexpr int NA = G >= 4 ? 1 : 4 / G;  // independent partial sums per head
@@ -123,27 +129,54 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
     for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int a = 0; a < NA; ++a) x[h][a] = 0.f;
-    const unsigned char *krow = ks + t * D * 2 + half * D;
-#pragma unroll
-    for (int i = 0; i < kNC; ++i) {
-        const int c = (i + lane) & (kNC - 1);
-        const uint4 raw = *reinterpret_cast<const uint4 *>(krow + c * 16);
-        const float2 k0 = E::to_float2(raw.x), k1 = E::to_float2(raw.y);
-        const float2 k2 = E::to_float2(raw.z), k3 = E::to_float2(raw.w);
+    const unsigned char *krow = ks + t * D * kEsz + half * (D / 2) * kEsz;
+    auto fma8 = [&](const float *k, int qchunk) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const float *qc = q_s + (h * 2 + half) * SimtQ<D>::kHalf + c * 12;
+            const float *qc = q_s + (h * 2 + half) * SimtQ<D>::kHalf + qchunk * 12;
             const float4 qa = *reinterpret_cast<const float4 *>(qc);
             const float4 qb = *reinterpret_cast<const float4 *>(qc + 4);
             float *a = x[h];
-            a[0 % NA] = fmaf(k0.x, qa.x, a[0 % NA]);
-            a[1 % NA] = fmaf(k0.y, qa.y, a[1 % NA]);
-            a[2 % NA] = fmaf(k1.x, qa.z, a[2 % NA]);
-            a[3 % NA] = fmaf(k1.y, qa.w, a[3 % NA]);
-            a[0 % NA] = fmaf(k2.x, qb.x, a[0 % NA]);
-            a[1 % NA] = fmaf(k2.y, qb.y, a[1 % NA]);
-            a[2 % NA] = fmaf(k3.x, qb.z, a[2 % NA]);
-            a[3 % NA] = fmaf(k3.y, qb.w, a[3 % NA]);
+            a[0 % NA] = fmaf(k[0], qa.x, a[0 % NA]);
+            a[1 % NA] = fmaf(k[1], qa.y, a[1 % NA]);
+            a[2 % NA] = fmaf(k[2], qa.z, a[2 % NA]);
+            a[3 % NA] = fmaf(k[3], qa.w, a[3 % NA]);
+            a[0 % NA] = fmaf(k[4], qb.x, a[0 % NA]);
+            a[1 % NA] = fmaf(k[5], qb.y, a[1 % NA]);
+            a[2 % NA] = fmaf(k[6], qb.z, a[2 % NA]);
+            a[3 % NA] = fmaf(k[7], qb.w, a[3 % NA]);
+        }
+    };
+    if constexpr (!kFp8) {
+        // 16-byte reads of 8 elements; rotated start per lane
+#pragma unroll
+        for (int i = 0; i < kNC; ++i) {
+            const int c = (i + lane) & (kNC - 1);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(krow + c * 16);
+            float k[8];
+            const float2 k0 = E::to_float2(raw.x), k1 = E::to_float2(raw.y);
+            const float2 k2 = E::to_float2(raw.z), k3 = E::to_float2(raw.w);
+            k[0] = k0.x; k[1] = k0.y; k[2] = k1.x; k[3] = k1.y;
+            k[4] = k2.x; k[5] = k2.y; k[6] = k3.x; k[7] = k3.y;
+            fma8(k, c);
+        }
+    } else {
+        // 16-byte reads of 16 E4M3 codes (two 8-element q chunks each)
+        constexpr int kNC16 = D / 32;
+#pragma unroll
+        for (int i = 0; i < kNC16; ++i) {
+            const int c = (i + lane) & (kNC16 - 1);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(krow + c * 16);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            float k[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 lo = e4m3x2_to_float2((uint16_t)(w[j] & 0xffffu));
+                const float2 hi = e4m3x2_to_float2((uint16_t)(w[j] >> 16));
+                k[4 * j] = lo.x; k[4 * j + 1] = lo.y; k[4 * j + 2] = hi.x; k[4 * j + 3] = hi.y;
+            }
+            fma8(k, 2 * c);
+            fma8(k + 8, 2 * c + 1);
         }
     }
 #pragma unroll
@@ -177,7 +210,21 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
 
     // P V: lane owns output dims [lane * kPV, lane * kPV + kPV)
     auto v_row = [&](int tok, float *vf) {
-        if constexpr (kPV == 4) {
+        if constexpr (kFp8) {
+            if constexpr (kPV == 4) {
+                const uint32_t raw = *reinterpret_cast<const uint32_t *>(vs + tok * D + lane * 4);
+                const float2 a = e4m3x2_to_float2((uint16_t)(raw & 0xffffu));
+                const float2 b = e4m3x2_to_float2((uint16_t)(raw >> 16));
+                vf[0] = a.x;
+                vf[1] = a.y;
+                vf[2] = b.x;
+                vf[3] = b.y;
+            } else {
+                const float2 a = e4m3x2_to_float2(*reinterpret_cast<const uint16_t *>(vs + tok * D + lane * 2));
+                vf[0] = a.x;
+                vf[1] = a.y;
+            }
+        } else if constexpr (kPV == 4) {
             const uint2 raw = *reinterpret_cast<const uint2 *>(vs + tok * D * 2 + lane * 8);
             const float2 a = E::to_float2(raw.x), b = E::to_float2(raw.y);
             vf[0] = a.x;

@@ -7,6 +7,11 @@ copy: that data stands for the prefill output of newly admitted sequences),
 then runs the step's ``pa_copy_blocks``, ``pa_reshape_and_cache`` and
 ``pa_decode`` calls through :mod:`.binding`.  torch provides the device
 memory and the stream; the three operations run in the library's kernels.
+
+Over an FP8 E4M3 cache (``scenario.kv_dtype == "fp8"``) the pools hold
+uint8 codes (NaN code 0x7F where nothing was written), admitted blocks enter
+through ``pa_reshape_and_cache_fp8`` like new tokens, and decode is
+``pa_decode_fp8`` with the scenario's scales.
 """
 from __future__ import annotations
 
@@ -31,25 +36,49 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+FP8_NAN_CODE = 0x7F
+ADMIT_CHUNK_BLOCKS = 4096  # admitted blocks per quantising write (bounds the staging copy)
+
+
 class DeviceSession:
     def __init__(self, scenario: Scenario, device: str = "cuda"):
         self.sc = scenario
         self.device = torch.device(device)
         d = scenario.dims
         self.dtype = TORCH_DTYPE[d.dtype]
+        self.fp8 = scenario.kv_dtype == "fp8"
         shape = (d.num_blocks, d.num_kv_heads, d.block_size, d.head_dim)
-        nan = np.array([NAN_BITS[d.dtype]], dtype=np.uint16).view(np.int16)[0]
-        self.k_cache = torch.full(shape, int(nan), dtype=torch.int16, device=self.device).view(self.dtype)
-        self.v_cache = torch.full(shape, int(nan), dtype=torch.int16, device=self.device).view(self.dtype)
+        if self.fp8:
+            self.k_cache = torch.full(shape, FP8_NAN_CODE, dtype=torch.uint8, device=self.device)
+            self.v_cache = torch.full(shape, FP8_NAN_CODE, dtype=torch.uint8, device=self.device)
+        else:
+            nan = np.array([NAN_BITS[d.dtype]], dtype=np.uint16).view(np.int16)[0]
+            self.k_cache = torch.full(shape, int(nan), dtype=torch.int16, device=self.device).view(self.dtype)
+            self.v_cache = torch.full(shape, int(nan), dtype=torch.int16, device=self.device).view(self.dtype)
         self._ws: Optional[torch.Tensor] = None
 
     # -- inputs ------------------------------------------------------------
     def admit(self, step: Step) -> None:
         if step.admit_ids.size == 0:
             return
-        ids = torch.from_numpy(step.admit_ids).to(self.device)
-        self.k_cache.index_copy_(0, ids, to_device(step.admit_k, self.sc.dims.dtype, self.device))
-        self.v_cache.index_copy_(0, ids, to_device(step.admit_v, self.sc.dims.dtype, self.device))
+        d = self.sc.dims
+        if not self.fp8:
+            ids = torch.from_numpy(step.admit_ids).to(self.device)
+            self.k_cache.index_copy_(0, ids, to_device(step.admit_k, d.dtype, self.device))
+            self.v_cache.index_copy_(0, ids, to_device(step.admit_v, d.dtype, self.device))
+            return
+        # FP8: every slot of each admitted block, token-major, through the quantising write
+        B = d.block_size
+        for c0 in range(0, step.admit_ids.size, ADMIT_CHUNK_BLOCKS):
+            sl = slice(c0, c0 + ADMIT_CHUNK_BLOCKS)
+            ids = torch.from_numpy(step.admit_ids[sl]).to(self.device)
+            key = to_device(step.admit_k[sl], d.dtype, self.device).transpose(1, 2).reshape(-1, d.num_kv_heads,
+                                                                                           d.head_dim)
+            val = to_device(step.admit_v[sl], d.dtype, self.device).transpose(1, 2).reshape(-1, d.num_kv_heads,
+                                                                                           d.head_dim)
+            slots = (ids[:, None] * B + torch.arange(B, device=self.device)[None, :]).reshape(-1)
+            pa.pa_reshape_and_cache_fp8(key.contiguous(), val.contiguous(), self.k_cache, self.v_cache, slots,
+                                        self.sc.k_scale, self.sc.v_scale)
 
     def decode_inputs(self, step: Step) -> Dict[str, torch.Tensor]:
         d = self.sc.dims
@@ -78,6 +107,13 @@ class DeviceSession:
             bm = torch.from_numpy(np.ascontiguousarray(step.block_mapping)).to(self.device)
             pa.pa_copy_blocks([self.k_cache], [self.v_cache], bm)
         for key, value, slots in self.write_inputs(step):
+            self.write(key, value, slots)
+
+    def write(self, key: torch.Tensor, value: torch.Tensor, slots: torch.Tensor) -> None:
+        if self.fp8:
+            pa.pa_reshape_and_cache_fp8(key, value, self.k_cache, self.v_cache, slots, self.sc.k_scale,
+                                        self.sc.v_scale)
+        else:
             pa.pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots)
 
     def decode(self, step: Step, partition_tokens: Optional[int] = None,
@@ -90,8 +126,12 @@ class DeviceSession:
         ws = self.workspace(pa.pa_decode_workspace_size(dims, maxlen, P))
         if out is None:
             out = torch.empty((d.num_seqs, d.num_heads, d.head_dim), dtype=self.dtype, device=self.device)
-        pa.pa_decode(out, inp["q"], self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"],
-                     self.sc.scale, d.num_kv_heads, maxlen, P, ws)
+        if self.fp8:
+            pa.pa_decode_fp8(out, inp["q"], self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"],
+                             self.sc.scale, self.sc.k_scale, self.sc.v_scale, d.num_kv_heads, maxlen, P, ws)
+        else:
+            pa.pa_decode(out, inp["q"], self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"],
+                         self.sc.scale, d.num_kv_heads, maxlen, P, ws)
         return out
 
     def run_step(self, step: Step, partition_tokens: Optional[int] = None) -> torch.Tensor:

@@ -134,6 +134,17 @@ class Scenario:
     partition_tokens: int = 0
     note: str = ""
     shared_blocks: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))
+    # KV cache element type: "" = the 16-bit dtype of the tokens, "fp8" =
+    # E4M3 codes with per-tensor scales (K = code * k_scale, V likewise).
+    # The step data stays 16-bit: admitted blocks and new tokens reach an
+    # FP8 cache through the quantising cache write on either side.
+    kv_dtype: str = ""
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+
+    @property
+    def kv_elem_bytes(self) -> int:
+        return 1 if self.kv_dtype == "fp8" else 2
 
 
 # --------------------------------------------------------------------------
@@ -362,16 +373,30 @@ def cow(seed: int = 4, num_prompts: int = 16, samples: int = 8, prefix: int = 10
                     shared_blocks=np.asarray(shared, np.int64))
 
 
+# Per-tensor FP8 scales for inputs in [-1, 1]: |x| / scale reaches 81 (K)
+# and 141 (V), inside E4M3's range (448).  Not powers of two, so the
+# division before rounding is inexact and both sides must round it alike.
+FP8_K_SCALE = 0.0123
+FP8_V_SCALE = 0.0071
+
+
+def with_fp8_cache(sc: Scenario, k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> Scenario:
+    """The same scenario over an FP8 E4M3 cache."""
+    return replace(sc, name=f"{sc.name}-fp8", kv_dtype="fp8", k_scale=float(np.float32(k_scale)),
+                   v_scale=float(np.float32(v_scale)),
+                   note=f"{sc.note}; FP8 E4M3 cache, k_scale {k_scale}, v_scale {v_scale}")
+
+
 SCENARIOS = {"tiny": tiny, "mha7b": mha7b, "gqa8b": gqa8b, "long70b": long70b, "cow": cow}
 CONFIG_ORDER = ["tiny", "mha7b", "gqa8b", "long70b", "cow"]
 
 
-def kv_bytes(step: Step, dims: Dims, unique: bool = False) -> int:
+def kv_bytes(step: Step, dims: Dims, unique: bool = False, elem_bytes: int = 2) -> int:
     """KV bytes a decode step must read: sum of context lengths x 2 (K and V)
-    x KV heads x head_dim x element size (2 bytes).  With ``unique``, blocks
-    shared by several sequences count once (whole blocks, partial tails as
-    their token count)."""
-    el = 2
+    x KV heads x head_dim x element size (2 bytes; 1 for an FP8 cache).  With
+    ``unique``, blocks shared by several sequences count once (whole blocks,
+    partial tails as their token count)."""
+    el = elem_bytes
     per_tok = 2 * dims.num_kv_heads * dims.head_dim * el
     if not unique:
         return int(step.context_lens.astype(np.int64).sum()) * per_tok

@@ -50,15 +50,21 @@ def compare_pools(dev, orc_ses: OracleSession, what: str) -> None:
     ids = np.asarray(pool.ids, dtype=np.int64)
     rows = pool.row_of[ids]
     idx = torch.from_numpy(ids).to(dev.k_cache.device)
+    fp8 = pool.dtype == "fp8"
     for name, cache, host in (("K", dev.k_cache, pool.k), ("V", dev.v_cache, pool.v)):
-        got = cache.view(torch.int16).index_select(0, idx).cpu().numpy().view(np.uint16)
+        if fp8:  # uint8 E4M3 codes; 0x7F (NaN) where nothing was written
+            got = cache.index_select(0, idx).cpu().numpy()
+            raw, nan = cache, 0x7F
+        else:
+            got = cache.view(torch.int16).index_select(0, idx).cpu().numpy().view(np.uint16)
+            raw = cache.view(torch.int16)
+            nan = int(np.array([NAN_BITS[orc_ses.sc.dims.dtype]], np.uint16).view(np.int16)[0])
         want = host[rows]
         bad = np.nonzero((got != want).reshape(len(ids), -1).any(axis=1))[0]
         assert bad.size == 0, f"{what}: {name} blocks differ at physical ids {ids[bad[:8]].tolist()}"
         mask = torch.ones(cache.shape[0], dtype=torch.bool, device=cache.device)
         mask[idx] = False
-        nan = int(np.array([NAN_BITS[orc_ses.sc.dims.dtype]], np.uint16).view(np.int16)[0])
-        untouched = cache.view(torch.int16)[mask]
+        untouched = raw[mask]
         assert bool((untouched == nan).all()), f"{what}: {name} bytes outside the written blocks changed"
 
 

@@ -436,8 +436,8 @@ def pin_e4m3_widen_every_code(orc):
 
 def pin_e4m3_quantize_matches_torch_in_range(orc):
     """Random values, every representable value and every midpoint between
-    neighbours (the tie cases) up to 448: same codes as torch's
-    round-to-nearest-even conversion."""
+    neighbours (the tie cases) up to 448, both signs: same codes as torch's
+    round-to-nearest-even conversion, the sign of zero included."""
     rng = np.random.default_rng(17)
     vals = e4m3_torch(np.arange(0, 0x7f, dtype=np.uint8))        # +0 .. 448
     mids = (vals[:-1] + vals[1:]) / 2
@@ -446,9 +446,9 @@ def pin_e4m3_quantize_matches_torch_in_range(orc):
     y = np.concatenate([y, -y])
     want = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     got = orc.quantize_e4m3(y)
-    zero = y == 0  # torch keeps the sign of zero; compare -0 and +0 by value
-    assert np.array_equal(got[~zero], want[~zero]), "quantisation differs from torch in range"
-    assert np.all(orc.widen_e4m3(got[zero]) == 0)
+    # exact, zeros included: -0.0 and negatives that round to zero give -0 (0x80)
+    assert np.array_equal(got, want), "quantisation differs from torch in range"
+    assert got[np.signbit(y) & (y == 0)].tolist() and np.all(got[np.signbit(y) & (y == 0)] == 0x80)
 
 
 def pin_e4m3_saturates_to_finite(orc):

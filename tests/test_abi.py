@@ -77,12 +77,21 @@ def test_workspace_plan(lib):
 @pytest.mark.parametrize("kw,status", [
     (dict(block_size=32), -4), (dict(head_dim=96), -4), (dict(num_heads=24, num_kv_heads=8), -4),
     (dict(num_heads=30), -3), (dict(dtype=7), -2), (dict(num_kv_heads=0), -3), (dict(num_seqs=-1), -3),
-    (dict(num_seqs=70000), -3),
+    (dict(num_seqs=70000), -3), (dict(kv_dtype=5), -2), (dict(dtype=0, kv_dtype=1), -2),
 ])
 def test_bad_dims_rejected(lib, kw, status):
     d = _dims(lib, **kw)
     assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, 0) == status
     assert lib.pa_last_error()
+
+
+def test_fp8_cache_plans_on_the_cuda_core_kernel(lib):
+    # group 4 / head_dim 128 would take the tensor-core kernel (1024-token
+    # partitions) over a 16-bit cache; an FP8 cache takes the CUDA-core one (512)
+    d = _dims(lib, kv_dtype=lib.PA_FP8_E4M3)
+    assert lib.pa_decode_num_partitions(d, 1024, 0) == 2
+    assert lib.pa_decode_num_partitions(d, 4096, 0) == 8
+    assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=lib.PA_BF16), 1024, 0) == 1
 
 
 def test_bad_partition_and_context(lib):
@@ -137,6 +146,33 @@ assert L.pa_copy_blocks(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctyp
 assert L.pa_copy_blocks(None, None, 0, None, 0, ctypes.byref(d), None) == 0
 assert L.pa_copy_blocks(None, None, 1, p, -1, ctypes.byref(d), None) == -3
 assert L.pa_device_error(None, None) == -1
+
+# FP8 E4M3 caches: entry point and kv_dtype must agree; scales must be positive
+f8 = dims(kv_dtype=lib.PA_FP8_E4M3)
+def decode_fp8(d, ptrs=good, ks=0.5, vs=0.5, maxlen=100):
+    out, q, k, v, bt, cl = ptrs
+    return L.pa_decode_fp8(out, q, k, v, bt, cl, ctypes.c_float(0.1), ctypes.c_float(ks), ctypes.c_float(vs), 8,
+                           ctypes.byref(d), maxlen, 0, None, 0, None)
+assert decode(f8, good, maxlen=100) == -2          # pa_decode on an FP8 cache
+assert "pa_decode_fp8" in lib.pa_last_error()
+assert decode_fp8(d) == -2                         # pa_decode_fp8 on a 16-bit cache
+assert decode_fp8(f8, ks=0.0) == -3
+assert decode_fp8(f8, vs=-1.0) == -3
+assert decode_fp8(f8, ks=float("inf")) == -3
+assert decode_fp8(f8, ks=float("nan")) == -3
+assert decode_fp8(f8, maxlen=2000) == -5           # split, no workspace
+assert decode_fp8(f8, ptrs=[None] + good[1:]) == -1
+assert decode_fp8(f8, ptrs=[ctypes.c_void_p(0x10008)] + good[1:]) == -7
+def rc8(d, key=p, ks=0.5, vs=0.5, n=4):
+    return L.pa_reshape_and_cache_fp8(key, p, p, p, p, n, ctypes.byref(d), ctypes.c_float(ks), ctypes.c_float(vs),
+                                      None)
+assert rc8(d) == -2                                # 16-bit cache
+assert L.pa_reshape_and_cache(p, p, p, p, p, 4, ctypes.byref(f8), None) == -2
+assert rc8(f8, ks=0.0) == -3
+assert rc8(f8, n=-1) == -3
+assert rc8(f8, key=None) == -1
+assert rc8(f8, key=ctypes.c_void_p(0x10004)) == -7
+assert rc8(f8, key=None, n=0) == 0
 print("host checks ok")
 """
 

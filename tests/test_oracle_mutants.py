@@ -69,6 +69,7 @@ MUTANTS = {
     "e4m3_exponent_bias": ("v = ldexp((double)(m + 8), e - 10);", "v = ldexp((double)(m + 8), e - 9);"),
     "e4m3_ties_to_odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
     "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "e4m3_zero_sign_dropped": ("(signbit(y) ? 0x80 : 0)", "(y < 0 ? 0x80 : 0)"),
     "fp8_k_scale_dropped": ("* (widen_e4m3(k_cache[row + d]) * k_scale);", "* widen_e4m3(k_cache[row + d]);"),
     "fp8_scales_swapped": ("o[d] += w * (widen_e4m3(v_cache[row + d]) * v_scale);",
                            "o[d] += w * (widen_e4m3(v_cache[row + d]) * k_scale);"),
