@@ -92,6 +92,9 @@ class Oracle:
         lib.oracle_reshape_and_cache_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32,
                                                      ctypes.c_float, ctypes.c_float]
         lib.oracle_reshape_and_cache_fp8.restype = ctypes.c_int
+        lib.oracle_paged_decode_ext.argtypes = [vp, vp, vp, vp, vp, vp, dbl, dbl, dbl, i32, i32, i32, i32, i32,
+                                                i32, i64, i32, i32, i32, i32]
+        lib.oracle_paged_decode_ext.restype = ctypes.c_int
         lib.oracle_quantize_e4m3_n.argtypes = [vp, vp, i64]
         lib.oracle_quantize_e4m3_n.restype = None
         lib.oracle_widen_e4m3_n.argtypes = [vp, vp, i64]
@@ -216,6 +219,35 @@ class Oracle:
                                                NB, _DTYPE_CODE[dtype])
         if rc != 0:
             raise OracleError(f"oracle_paged_decode_fp8 returned {rc}")
+        return out
+
+    def paged_decode_ext(self, q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype: str,
+                         q_len: int = 1, window: int = 0, k_scale: float = 1.0, v_scale: float = 1.0) -> np.ndarray:
+        """Multi-token / sliding-window decode: q and the result are
+        ``[S, q_len, H, D]``; query i of sequence s sits at position
+        ``context_lens[s] - q_len + i`` and attends causally to the ``window``
+        most recent positions (all when 0).  The caches hold 16-bit bit
+        patterns (uint16) or E4M3 codes (uint8); K and V are scaled by
+        ``k_scale`` / ``v_scale``."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        if k_cache.dtype not in (np.uint16, np.uint8) or v_cache.dtype != k_cache.dtype:
+            raise OracleError("caches must both be uint16 (16-bit) or uint8 (E4M3)")
+        k_cache = np.ascontiguousarray(k_cache)
+        v_cache = np.ascontiguousarray(v_cache)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, QL, H, D = q.shape
+        NB, Hk, B, D2 = k_cache.shape
+        if QL != q_len or D2 != D or v_cache.shape != k_cache.shape or bt.shape[0] != S or cl.shape != (S,):
+            raise OracleError("shape mismatch")
+        MB = bt.shape[1] if bt.ndim == 2 else 0
+        out = np.zeros((S, q_len, H, D), dtype=np.float64)
+        rc = self._lib.oracle_paged_decode_ext(_p(out), _p(q), _p(k_cache), _p(v_cache), _p(bt), _p(cl),
+                                               float(scale), float(k_scale), float(v_scale), S, H, Hk, D, B, MB,
+                                               NB, _DTYPE_CODE[dtype], int(k_cache.dtype == np.uint8), int(q_len),
+                                               int(window))
+        if rc != 0:
+            raise OracleError(f"oracle_paged_decode_ext returned {rc}")
         return out
 
     def reshape_and_cache_fp8(self, k_cache, v_cache, key, value, slot_mapping, dtype: str, k_scale: float,

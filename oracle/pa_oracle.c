@@ -448,3 +448,119 @@ int oracle_reshape_and_cache_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint1
     }
     return ORC_OK;
 }
+
+/*
+ * Multi-token and sliding-window decode (variants of the same path: a
+ * sliding-window mask over the same block stream, which "vLLM PagedAttention
+ * 大模型推理架构深度实战" section 7.2 recommends for long contexts, and several
+ * query tokens per sequence, as the large model's parallel verification of
+ * draft tokens in speculative decoding needs, the same page's section 九
+ * item 2).  Readings, where the page gives no formula:
+ *   - the q_len query tokens of sequence s are its last q_len tokens, whose
+ *     K/V are already in the cache: query i sits at position
+ *     p_i = context_lens[s] - q_len + i and attends causally to j <= p_i;
+ *   - a window of W > 0 tokens keeps the W most recent positions including
+ *     the query's own: j >= p_i - W + 1 (W = 0: no window);
+ *   - a query with no position to attend to (p_i < 0) gets a zero row.
+ * For sequence s, query token i, query head h (KV head kvh = h / group),
+ * lo_i = W > 0 ? max(0, p_i - W + 1) : 0:
+ *   x_j = scale * sum_d q[s, i, h, d] * K_s[j, d] * k_scale    (lo_i <= j <= p_i)
+ *   out[s, i, h, :] = sum_j softmax(x)_j * V_s[j, :] * v_scale
+ * K_s / V_s through the block table as in oracle_paged_decode; the cache
+ * holds 16-bit elements of `dtype` (kv_fp8 = 0) or E4M3 codes (kv_fp8 = 1).
+ * q and out are [num_seqs, q_len, num_heads, head_dim].  Only the blocks
+ * holding positions lo_i .. p_i are read (table entries of blocks before the
+ * window are never touched).
+ */
+int oracle_paged_decode_ext(double *out, const uint16_t *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, const int32_t *context_lens, double scale,
+                            double k_scale, double v_scale, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype, int32_t kv_fp8,
+                            int32_t q_len, int32_t window) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return ORC_ERR_ARG;
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq < 0 || num_blocks <= 0 || q_len <= 0 || window < 0)
+        return ORC_ERR_ARG;
+    if (num_heads % num_kv_heads != 0) return ORC_ERR_ARG;
+    if (dtype != ORC_F16 && dtype != ORC_BF16) return ORC_ERR_ARG;
+    const uint16_t *k16 = (const uint16_t *)k_cache, *v16 = (const uint16_t *)v_cache;
+    const uint8_t *k8 = (const uint8_t *)k_cache, *v8 = (const uint8_t *)v_cache;
+
+    /* Every block id that will be read must lie in the pool. */
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t n = context_lens[s];
+        if (n < 0 || (int64_t)n > (int64_t)max_blocks_per_seq * block_size) return ORC_ERR_RANGE;
+        for (int32_t i = 0; i < q_len; ++i) {
+            int32_t hi = n - q_len + i;
+            if (hi < 0) continue;
+            int32_t lo = window > 0 && hi - window + 1 > 0 ? hi - window + 1 : 0;
+            for (int32_t bi = lo / block_size; bi <= hi / block_size; ++bi) {
+                int32_t b = block_tables[(int64_t)s * max_blocks_per_seq + bi];
+                if (b < 0 || (int64_t)b >= num_blocks) return ORC_ERR_RANGE;
+            }
+        }
+    }
+
+    const int32_t group = num_heads / num_kv_heads;
+    const int64_t rows = (int64_t)num_seqs * q_len * num_heads;
+    int status = ORC_OK;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int32_t s = (int32_t)(r / ((int64_t)q_len * num_heads));
+        const int32_t i = (int32_t)(r / num_heads % q_len);
+        const int32_t h = (int32_t)(r % num_heads);
+        const int32_t kvh = h / group;
+        const int32_t hi = context_lens[s] - q_len + i;
+        double *o = out + r * head_dim;
+        for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;
+        if (hi < 0) continue;
+        const int32_t lo = window > 0 && hi - window + 1 > 0 ? hi - window + 1 : 0;
+        const int32_t n = hi - lo + 1;
+
+        double *x = (double *)malloc(sizeof(double) * (size_t)n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        if (!x || !qd) {
+            free(x);
+            free(qd);
+#pragma omp atomic write
+            status = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int32_t d = 0; d < head_dim; ++d) qd[d] = widen(q[r * head_dim + d], dtype);
+
+        /* logits of positions lo .. hi through the block table */
+        for (int32_t j = lo; j <= hi; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double dot = 0.0;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                double kv = kv_fp8 ? widen_e4m3(k8[row + d]) : widen(k16[row + d], dtype);
+                dot += qd[d] * (kv * k_scale);
+            }
+            x[j - lo] = scale * dot;
+        }
+        /* softmax (max-subtracted) and the weighted sum of V */
+        double m = -INFINITY;
+        for (int32_t j = 0; j < n; ++j)
+            if (x[j] > m) m = x[j];
+        double z = 0.0;
+        for (int32_t j = 0; j < n; ++j) {
+            x[j] = exp(x[j] - m);
+            z += x[j];
+        }
+        for (int32_t j = lo; j <= hi; ++j) {
+            int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + j / block_size];
+            int64_t row = ((blk * num_kv_heads + kvh) * block_size + j % block_size) * head_dim;
+            double w = x[j - lo] / z;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                double vv = kv_fp8 ? widen_e4m3(v8[row + d]) : widen(v16[row + d], dtype);
+                o[d] += w * (vv * v_scale);
+            }
+        }
+        free(x);
+        free(qd);
+    }
+    return status;
+}

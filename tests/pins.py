@@ -513,4 +513,143 @@ def pin_brute_force_tiny(orc):
     assert_close(out, ref, 1e-13, "oracle vs brute force")
 
 
+
+# ---------------------------------------------------------------------------
+# multi-token / sliding-window decode pins
+# ---------------------------------------------------------------------------
+def ext_q(rng, S, q_len, H, D, dtype):
+    return rand_bits(rng, (S, q_len, H, D), dtype)
+
+
+def masked_sdpa(q_bits, k_bits, v_bits, L, q_len, window, scale, dtype):
+    """torch float64 SDPA for one sequence with an explicit boolean mask:
+    q [q_len, H, D], k/v [L, Hk, D]; query i sees positions
+    max(0, p - W + 1) .. p with p = L - q_len + i (all up to p when W = 0).
+    Rows with p < 0 are zero."""
+    H = q_bits.shape[1]
+    out = np.zeros((q_len, H, q_bits.shape[2]))
+    pos = np.arange(L)
+    mask = np.zeros((q_len, L), dtype=bool)
+    for i in range(q_len):
+        p = L - q_len + i
+        lo = max(0, p - window + 1) if window > 0 else 0
+        mask[i] = (pos <= p) & (pos >= lo)
+    live = mask.any(axis=1)
+    if L == 0 or not live.any():
+        return out
+    q = torch.from_numpy(widen(q_bits, dtype)).permute(1, 0, 2)[None]          # [1, H, q_len, D]
+    k = torch.from_numpy(widen(k_bits, dtype)).permute(1, 0, 2)[None]          # [1, Hk, L, D]
+    v = torch.from_numpy(widen(v_bits, dtype)).permute(1, 0, 2)[None]
+    m = torch.from_numpy(mask)
+    m[~torch.from_numpy(live)] = True  # keep torch finite on dead rows; they are overwritten
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale,
+                                                         enable_gqa=q.shape[1] != k.shape[1])
+    o = o[0].permute(1, 0, 2).numpy()
+    out[live] = o[live]
+    return out
+
+
+def pin_ext_matches_masked_sdpa(orc):
+    """Multi-token and sliding-window decode equal torch SDPA with the
+    causal-window mask written out, for q_len 1-3, windows 0/1/7/16/33, GQA,
+    lengths below q_len (zero rows) through 100."""
+    rng = np.random.default_rng(71)
+    lens = [1, 2, 5, 16, 17, 40, 100]
+    for dtype in ("f16", "bf16"):
+        p = Paged(rng, lens, 8, 2, 16, dtype)
+        for q_len in (1, 3):
+            q = ext_q(rng, len(lens), q_len, 8, 16, dtype)
+            for window in (0, 1, 7, 16, 33):
+                got = orc.paged_decode_ext(q, p.k_cache, p.v_cache, p.tables, p.lens, 0.3, dtype, q_len, window)
+                for s, L in enumerate(lens):
+                    want = masked_sdpa(q[s], p.ks[s], p.vs[s], L, q_len, window, 0.3, dtype)
+                    assert_close(got[s], want, 1e-12, f"ext {dtype} q_len={q_len} W={window} L={L}")
+
+
+def pin_ext_reduces_to_decode(orc):
+    """q_len 1 without a window is plain decode; a window at least as long as
+    the context changes nothing."""
+    rng = np.random.default_rng(72)
+    lens = [1, 16, 33, 300]
+    p = Paged(rng, lens, 8, 4, 32, "bf16")
+    base = p.run(orc, 0.2)
+    for window in (0, 300, 1000):
+        got = orc.paged_decode_ext(p.q[:, None], p.k_cache, p.v_cache, p.tables, p.lens, 0.2, "bf16", 1, window)
+        assert np.array_equal(got[:, 0], base), f"window {window}"
+
+
+def pin_ext_window_one_returns_own_value(orc):
+    """A window of one token: each query returns V at its own position."""
+    rng = np.random.default_rng(73)
+    lens = [3, 16, 17, 50]
+    p = Paged(rng, lens, 4, 2, 16, "f16")
+    q = ext_q(rng, len(lens), 3, 4, 16, "f16")
+    got = orc.paged_decode_ext(q, p.k_cache, p.v_cache, p.tables, p.lens, 0.5, "f16", 3, 1)
+    for s, L in enumerate(lens):
+        for i in range(3):
+            want = widen(p.vs[s][L - 3 + i], "f16")       # [Hk, D]
+            assert np.array_equal(got[s, i], np.repeat(want, 2, axis=0)), f"s={s} i={i}"
+
+
+def pin_ext_query_i_is_a_truncated_decode(orc):
+    """Query i of a multi-token call equals a single-query call whose context
+    ends at that query's position (with and without a window)."""
+    rng = np.random.default_rng(74)
+    lens = [4, 20, 64, 129]
+    p = Paged(rng, lens, 8, 8, 32, "bf16")
+    q = ext_q(rng, len(lens), 4, 8, 32, "bf16")
+    for window in (0, 10):
+        got = orc.paged_decode_ext(q, p.k_cache, p.v_cache, p.tables, p.lens, 0.25, "bf16", 4, window)
+        for i in range(4):
+            lens_i = p.lens - 4 + i + 1
+            one = orc.paged_decode_ext(np.ascontiguousarray(q[:, i:i + 1]), p.k_cache, p.v_cache, p.tables, lens_i,
+                                       0.25, "bf16", 1, window)
+            assert np.array_equal(got[:, i], one[:, 0]), f"query {i} window {window}"
+
+
+def pin_ext_scales_and_fp8(orc):
+    """K and V scales multiply the cache elements: a 16-bit cache scaled by
+    powers of two equals the pre-scaled cache, and E4M3 codes equal their
+    exactly widened 16-bit values."""
+    rng = np.random.default_rng(75)
+    lens = [5, 31, 70]
+    p = Paged(rng, lens, 4, 2, 16, "f16")
+    q = ext_q(rng, len(lens), 2, 4, 16, "f16")
+    got = orc.paged_decode_ext(q, p.k_cache, p.v_cache, p.tables, p.lens, 0.3, "f16", 2, 9, k_scale=4.0,
+                               v_scale=0.5)
+    k4 = narrow(widen(p.k_cache, "f16") * 4.0, "f16")
+    v5 = narrow(widen(p.v_cache, "f16") * 0.5, "f16")
+    want = orc.paged_decode_ext(q, k4, v5, p.tables, p.lens, 0.3, "f16", 2, 9)
+    assert np.array_equal(got, want), "scales are not applied to the elements"
+    NB, Hk, B, D = p.k_cache.shape
+    kc = rng.integers(0, 256, size=(NB, Hk, B, D), dtype=np.uint8)
+    kc[(kc & 0x7F) == 0x7F] = 0x38
+    vc = np.roll(kc, 1, axis=0)
+    got8 = orc.paged_decode_ext(q, kc, vc, p.tables, p.lens, 0.01, "f16", 2, 9, k_scale=0.25, v_scale=2.0)
+    k16 = narrow(e4m3_torch(kc) * 0.25, "f16")
+    v16 = narrow(e4m3_torch(vc) * 2.0, "f16")
+    want8 = orc.paged_decode_ext(q, k16, v16, p.tables, p.lens, 0.01, "f16", 2, 9)
+    assert np.array_equal(got8, want8), "E4M3 ext decode differs from the widened 16-bit one"
+
+
+def pin_ext_reads_no_block_before_the_window(orc):
+    """Table entries of blocks wholly before every query's window are never
+    read (they may hold anything); without the window the same entries are."""
+    rng = np.random.default_rng(76)
+    lens = [100, 64]
+    p = Paged(rng, lens, 4, 4, 16, "f16")
+    q = ext_q(rng, 2, 2, 4, 16, "f16")
+    want = orc.paged_decode_ext(q, p.k_cache, p.v_cache, p.tables, p.lens, 0.3, "f16", 2, 20)
+    t = p.tables.copy()
+    t[0, :4] = -1      # sequence 0: window covers positions 79..99 -> blocks 4..6
+    t[1, :2] = 10 ** 6  # sequence 1: positions 43..63 -> blocks 2..3
+    got = orc.paged_decode_ext(q, p.k_cache, p.v_cache, t, p.lens, 0.3, "f16", 2, 20)
+    assert np.array_equal(got, want)
+    from oracle import OracleError
+    try:
+        orc.paged_decode_ext(q, p.k_cache, p.v_cache, t, p.lens, 0.3, "f16", 2, 0)
+    except OracleError:
+        return
+    raise AssertionError("entries inside the attended range must be checked")
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -75,6 +75,16 @@ MUTANTS = {
                            "o[d] += w * (widen_e4m3(v_cache[row + d]) * k_scale);"),
     "fp8_write_scale_multiplied": ("quantize_e4m3((float)widen(key[src + d], dtype) / k_scale, &tab)",
                                    "quantize_e4m3((float)widen(key[src + d], dtype) * k_scale, &tab)"),
+    "ext_window_off_by_one": ("const int32_t lo = window > 0 && hi - window + 1 > 0 ? hi - window + 1 : 0;",
+                              "const int32_t lo = window > 0 && hi - window > 0 ? hi - window : 0;"),
+    "ext_window_ignored": ("const int32_t lo = window > 0 && hi - window + 1 > 0 ? hi - window + 1 : 0;",
+                           "const int32_t lo = 0;"),
+    "ext_causal_shift": ("const int32_t hi = context_lens[s] - q_len + i;",
+                         "const int32_t hi = context_lens[s] - q_len + i - (i > 0);"),
+    "ext_first_query_row_for_all": ("qd[d] = widen(q[r * head_dim + d], dtype);",
+                                    "qd[d] = widen(q[(r - (int64_t)i * num_heads) * head_dim + d], dtype);"),
+    "ext_k_scale_dropped": ("dot += qd[d] * (kv * k_scale);", "dot += qd[d] * kv;"),
+    "ext_v_scale_dropped": ("o[d] += w * (vv * v_scale);", "o[d] += w * vv;"),
     "zero_length_not_zeroed": ("for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;\n        if (n == 0) continue;",
                                "if (n == 0) { o[0] = 1.0; continue; }\n        "
                                "for (int32_t d = 0; d < head_dim; ++d) o[d] = 0.0;"),
