@@ -48,8 +48,10 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha7b", choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "swap"],
-                    help="decode scenario, or 'swap' for pa_swap_blocks device <-> pinned host throughput")
+    ap.add_argument("--workload", default="mha7b",
+                    choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "spec8b", "window70b", "swap"],
+                    help="decode scenario (spec8b: 4 query tokens per sequence; window70b: 4096-token sliding "
+                         "window), or 'swap' for pa_swap_blocks device <-> pinned host throughput")
     ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
     ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
@@ -261,9 +263,14 @@ def run_ours(args):
     bm = torch.from_numpy(np.ascontiguousarray(st.block_mapping)).to(device) if st.block_mapping.size else None
     maxlen = st.max_context_len
     dims = pa.dims_of(inp["q"], dev.k_cache, inp["block_tables"])
-    nparts = pa.pa_decode_num_partitions(dims, maxlen, P)
-    ws = dev.workspace(pa.pa_decode_workspace_size(dims, maxlen, P))
-    out = torch.empty((d.num_seqs, d.num_heads, d.head_dim), dtype=dev.dtype, device=device)
+    if sc.ext:
+        ws_bytes = dev.ext_workspace_bytes(inp, maxlen, P)
+        nparts = "split" if ws_bytes else 1
+    else:
+        nparts = pa.pa_decode_num_partitions(dims, maxlen, P)
+        ws_bytes = pa.pa_decode_workspace_size(dims, maxlen, P)
+    ws = dev.workspace(ws_bytes)
+    out = torch.empty_like(inp["q"])
     stream = torch.cuda.current_stream(device)
 
     def write(key, value, slots):
@@ -274,7 +281,9 @@ def run_ours(args):
             pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
 
     def decode(q, bt, cl):
-        if fp8:
+        if sc.ext:
+            dev.decode_ext({"q": q, "block_tables": bt, "context_lens": cl}, maxlen, P, out, stream=stream)
+        elif fp8:
             pa.pa_decode_fp8(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.k_scale, sc.v_scale,
                              d.num_kv_heads, maxlen, P, ws, stream=stream)
         else:
@@ -292,7 +301,7 @@ def run_ours(args):
         if e1 is not None:
             e1.record(stream)
 
-    launches_per_step = (1 if bm is not None else 0) + len(writes) + (2 if nparts > 1 else 1)
+    launches_per_step = (1 if bm is not None else 0) + len(writes) + (2 if ws_bytes else 1)
 
     for _ in range(args.warmup):
         step()
@@ -375,9 +384,9 @@ def run_ours(args):
 
     # Algorithmic bytes: KV of the referenced tokens; blocks shared by several
     # sequences (copy-on-write prefixes) count once, as the pool holds them once.
-    kv_logical = W.kv_bytes(st, d, elem_bytes=sc.kv_elem_bytes)
+    kv_logical = W.kv_bytes(st, d, elem_bytes=sc.kv_elem_bytes, q_len=sc.q_len, window=sc.window)
     kv = W.kv_bytes(st, d, unique=True, elem_bytes=sc.kv_elem_bytes) if args.workload == "cow" else kv_logical
-    algo = kv + W.qo_bytes(d)
+    algo = kv + W.qo_bytes(d, sc.q_len)
     peak, peak_kind = measured_hbm_peak()
     achieved = algo / (dec_avg_ms / 1e3) / 1e9
     traffic = ncu_traffic(args.workload + ("-fp8" if fp8 else ""), units=float(st.context_lens.sum()))
@@ -398,16 +407,17 @@ def run_ours(args):
                    "seq_len": "per-sequence, " + f"mean {float(st.context_lens.mean()):.0f}, "
                               f"max {int(st.context_lens.max())}",
                    "partition_tokens": P, "num_partitions": nparts,
+                   **({"q_len": sc.q_len, "window": sc.window} if sc.ext else {}),
                    "parallelism": f"{world} independent batches (one per GPU, no data-path collective)",
                    "l2": f"inputs larger than L2: {kv / 1e9:.2f} GB of KV read per step vs 126 MB L2",
                    "kv_bytes_per_step": kv, "kv_bytes_logical_per_step": kv_logical,
                    "algorithmic_bytes_per_step": algo},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": ("pa_decode_fp8" if fp8 else "pa_decode") +
-                               (" (decode kernel + log-sum-exp merge)" if nparts > 1 else ""),
+                     "kernel": ("pa_decode_ext" if sc.ext else "pa_decode_fp8" if fp8 else "pa_decode") +
+                               (" (decode kernel + log-sum-exp merge)" if ws_bytes else ""),
                      "kernel_ms": dec_avg_ms, "frac_of_8000": achieved / 8000.0,
-                     "effective_gbs_logical": (kv_logical + W.qo_bytes(d)) / (dec_avg_ms / 1e3) / 1e9},
+                     "effective_gbs_logical": (kv_logical + W.qo_bytes(d, sc.q_len)) / (dec_avg_ms / 1e3) / 1e9},
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,

@@ -8,6 +8,8 @@
  *   pa_copy_blocks        copy-on-write duplication of shared blocks
  *   pa_swap_blocks        block copies between device and host pools (preemption)
  *   pa_decode_fp8, pa_reshape_and_cache_fp8   the same over FP8 E4M3 caches
+ *   pa_decode_ext         several query tokens per sequence and/or a sliding
+ *                         window, over a 16-bit or FP8 cache
  *   pa_decode             single-query attention of every sequence over its
  *                         cached tokens, gathered through its block table
  *
@@ -197,6 +199,48 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
 pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
                                    const int64_t *slot_mapping, int32_t num_tokens, const pa_dims *dims,
                                    float k_scale, float v_scale, void *stream);
+
+/*
+ * Options of pa_decode_ext.  q_len query tokens per sequence (speculative
+ * verification: "vLLM PagedAttention 大模型推理架构深度实战" section 九 item 2),
+ * a sliding window (the same page, section 7.2, recommends it for long
+ * contexts) and per-tensor scales of the cached elements.
+ */
+typedef struct pa_decode_opts {
+    int32_t q_len;  /* >= 1; group * q_len <= 16 (group = num_heads / num_kv_heads) */
+    int32_t window; /* >= 0 tokens; 0 = no window */
+    float k_scale;  /* K element = stored value * k_scale; finite, > 0 (1 for a plain cache) */
+    float v_scale;  /* V element = stored value * v_scale; finite, > 0 */
+} pa_decode_opts;
+
+/* Workspace bytes pa_decode_ext needs (0 = none), (size_t)-1 for invalid
+ * dims or options. */
+size_t pa_decode_ext_workspace_size(const pa_dims *dims, const pa_decode_opts *opts, int32_t max_context_len,
+                                    int32_t partition_tokens);
+
+/*
+ * Multi-token / sliding-window decode over a 16-bit or FP8 E4M3 cache
+ * (dims->kv_dtype).  q and out are [num_seqs, q_len, num_heads, head_dim] in
+ * dims->dtype.  The q_len query tokens of sequence s are its last q_len
+ * tokens, already written to the cache: query i sits at position
+ * p = context_lens[s] - q_len + i and attends to positions j with
+ *     lo <= j <= p,   lo = window > 0 ? max(0, p - window + 1) : 0,
+ *     out[s, i, h, :] = sum_j softmax_j(scale * q[s, i, h, :] . K_s[j] * k_scale)
+ *                       * V_s[j] * v_scale
+ * (a query with p < 0 gets a zero row).  Only the blocks holding attended
+ * positions are read: table entries of blocks before a sequence's window
+ * may hold anything.  With q_len = 1, window = 0 and unit scales the result
+ * is pa_decode's.  max_context_len bounds context_lens as in pa_decode; the
+ * workspace is pa_decode_ext_workspace_size bytes.  Errors: those of
+ * pa_decode, plus PA_ERR_NULL for opts, PA_ERR_SHAPE for q_len < 1,
+ * window < 0 or a scale that is not finite and positive, PA_ERR_UNSUPPORTED
+ * for group * q_len > 16.
+ */
+pa_status pa_decode_ext(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens, float scale,
+                        int32_t num_kv_heads, const pa_dims *dims, const pa_decode_opts *opts,
+                        int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                        size_t workspace_bytes, void *stream);
 
 /*
  * Cache write (ybb.press section 六, "write into the KV cache block").

@@ -157,12 +157,35 @@ class OracleSession:
         if seqs is not None:
             seqs = np.asarray(seqs, dtype=np.int64)
             q, bt, cl = q[seqs], bt[seqs], cl[seqs]
+        q_len, window = getattr(self.sc, "q_len", 1), getattr(self.sc, "window", 0)
+        if q_len != 1 or window != 0:
+            rel = self.relabel_attended(bt, cl, q_len, window)
+            k, v = self.pool.view()
+            q4 = q if q.ndim == 4 else q[:, None]
+            out = self.orc.paged_decode_ext(q4, k, v, rel, cl, self.sc.scale, d.dtype, q_len, window,
+                                            self.sc.k_scale, self.sc.v_scale)
+            return out if q.ndim == 4 else out[:, 0]
         rel = self.pool.relabel_tables(bt, cl, d.block_size)
         k, v = self.pool.view()
         if self.fp8:
             return self.orc.paged_decode_fp8(q, k, v, rel, cl, self.sc.scale, self.sc.k_scale, self.sc.v_scale,
                                              d.dtype)
         return self.orc.paged_decode(q, k, v, rel, cl, self.sc.scale, d.dtype)
+
+    def relabel_attended(self, block_tables, context_lens, q_len: int, window: int) -> np.ndarray:
+        """Relabel only the entries of blocks some query attends to; entries
+        before a sequence's window become -1 (the oracle never reads them)."""
+        B = self.sc.dims.block_size
+        bt = np.asarray(block_tables, dtype=np.int64)
+        out = np.full(bt.shape, -1, dtype=np.int32)
+        for s in range(bt.shape[0]):
+            L = int(context_lens[s])
+            nb = -(-L // B)
+            lo = max(0, L - q_len - window + 1) if window > 0 else 0
+            first = lo // B
+            if nb > first:
+                out[s, first:nb] = self.pool.rows(bt[s, first:nb])
+        return out
 
     def run_step(self, step, seqs: Optional[np.ndarray] = None) -> np.ndarray:
         self.apply_cache_ops(step)

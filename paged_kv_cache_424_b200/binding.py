@@ -28,8 +28,9 @@ FP8_CACHE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
 # The C entry points declared in include/pa.h, in declaration order.
 EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_decode_noalloc",
-           "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks",
-           "pa_last_error", "pa_device_error", "pa_version"]
+           "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_decode_ext_workspace_size", "pa_decode_ext",
+           "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_last_error", "pa_device_error",
+           "pa_version"]
 
 
 class LibraryMissing(RuntimeError):
@@ -46,6 +47,11 @@ class pa_dims(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
                 ("num_blocks", ctypes.c_int64), ("dtype", ctypes.c_int32), ("kv_dtype", ctypes.c_int32)]
+
+
+class pa_decode_opts(ctypes.Structure):
+    _fields_ = [("q_len", ctypes.c_int32), ("window", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
 
 
 def _load(path: str = LIB_PATH):
@@ -67,6 +73,11 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_fp8.restype = ctypes.c_int
     lib.pa_reshape_and_cache_fp8.argtypes = [vp, vp, vp, vp, vp, i32, dp, f32, f32, vp]
     lib.pa_reshape_and_cache_fp8.restype = ctypes.c_int
+    op = ctypes.POINTER(pa_decode_opts)
+    lib.pa_decode_ext_workspace_size.argtypes = [dp, op, i32, i32]
+    lib.pa_decode_ext_workspace_size.restype = u64
+    lib.pa_decode_ext.argtypes = [vp, vp, vp, vp, vp, vp, f32, i32, dp, op, i32, i32, vp, u64, vp]
+    lib.pa_decode_ext.restype = ctypes.c_int
     lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, dp, vp]
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
@@ -224,6 +235,44 @@ def pa_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_c
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = LIB.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
                            float(scale), float(k_scale), float(v_scale), int(num_kv_heads), ctypes.byref(dims),
+                           int(max_context_len), int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st)
+    return out
+
+
+def pa_decode_ext_workspace_size(dims: pa_dims, opts: pa_decode_opts, max_context_len: int,
+                                 partition_tokens: int = 0) -> int:
+    n = LIB.pa_decode_ext_workspace_size(ctypes.byref(dims), ctypes.byref(opts), int(max_context_len),
+                                         int(partition_tokens))
+    if n == ctypes.c_size_t(-1).value:
+        raise PagedAttentionError(-3, pa_last_error())
+    return int(n)
+
+
+def ext_dims(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) -> pa_dims:
+    """dims of a [S, q_len, H, D] query batch."""
+    S, QL, H, D = q.shape
+    return dims_of(q.view(S, QL * H, D)[:, :H], k_cache, block_tables)
+
+
+def pa_decode_ext(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
+                  max_context_len: int, q_len: int = 1, window: int = 0, k_scale: float = 1.0, v_scale: float = 1.0,
+                  partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Multi-token / sliding-window decode: q and out are [S, q_len, H, D];
+    query i of sequence s sits at position context_lens[s] - q_len + i and
+    attends to its `window` most recent positions (all when 0).  The caches
+    may be 16-bit or FP8 E4M3 (uint8 / float8_e4m3fn)."""
+    _need_cuda(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if q.dim() != 4 or q.shape[1] != q_len or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, q_len, num_heads, head_dim]")
+    dims = ext_dims(q, k_cache, block_tables)
+    opts = pa_decode_opts(int(q_len), int(window), float(k_scale), float(v_scale))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = LIB.pa_decode_ext(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                           float(scale), int(num_kv_heads), ctypes.byref(dims), ctypes.byref(opts),
                            int(max_context_len), int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
     _check(st)
     return out

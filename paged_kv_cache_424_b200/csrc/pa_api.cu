@@ -73,7 +73,15 @@ struct Plan {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl) {
+// Rows per KV head (group x query tokens) rounded up to a built capacity.
+int row_capacity(int rows) {
+    int c = 1;
+    while (c < rows) c <<= 1;
+    return c;
+}
+
+pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
+                    int32_t q_len = 1, int32_t window = 0) {
     if (max_context_len < 0) return fail(PA_ERR_SHAPE, "max_context_len %d < 0", max_context_len);
     if ((int64_t)max_context_len > (int64_t)d->max_blocks_per_seq * d->block_size)
         return fail(PA_ERR_SHAPE, "max_context_len %d exceeds max_blocks_per_seq * block_size = %lld", max_context_len,
@@ -82,19 +90,26 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
                     partition_tokens, kMaxPartitionTokens);
     const int g = d->num_heads / d->num_kv_heads;
-    const bool tc = !kv_fp8(d) && pa::decode_tc_supported(d->head_dim, g, d->num_blocks, d->num_kv_heads);
+    const int rows = row_capacity(g * q_len);
+    const bool tc = !kv_fp8(d) && pa::decode_tc_supported(d->head_dim, rows, d->num_blocks, d->num_kv_heads);
     const int P = partition_tokens != 0 ? partition_tokens : tc ? kAutoPartitionTc : kAutoPartitionSimt;
-    const int ctx_blocks = (max_context_len + 15) / 16;
+    int ctx_blocks = (max_context_len + 15) / 16;
+    if (window > 0) {
+        // attended positions of a sequence span at most window + q_len - 1
+        // tokens, which may straddle one more block boundary
+        const int64_t span_blocks = ((int64_t)window + q_len - 1 + 15) / 16 + 1;
+        if (span_blocks < ctx_blocks) ctx_blocks = (int)span_blocks;
+    }
     int part_blocks = P / 16;
     const int max_parts = ctx_blocks == 0 ? 1 : (ctx_blocks + part_blocks - 1) / part_blocks;
     if (max_parts == 1) part_blocks = ctx_blocks > 0 ? ctx_blocks : 1;  // one partition: size it to the context
     pl->part_blocks = part_blocks;
     pl->max_parts = max_parts;
     if (max_parts > 1) {
-        const size_t rows = (size_t)d->num_seqs * d->num_heads * max_parts;
-        pl->o_bytes = align_up(rows * d->head_dim * sizeof(float), 256);
+        const size_t wrows = (size_t)d->num_seqs * q_len * d->num_heads * max_parts;
+        pl->o_bytes = align_up(wrows * d->head_dim * sizeof(float), 256);
         pl->lse_off = pl->o_bytes;
-        pl->ws_bytes = pl->o_bytes + align_up(rows * sizeof(float), 256);
+        pl->ws_bytes = pl->o_bytes + align_up(wrows * sizeof(float), 256);
     }
     return PA_OK;
 }
@@ -104,12 +119,13 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
 pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *block_tables, const int32_t *context_lens, float scale, float k_scale,
                       float v_scale, int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
-                      int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream) {
+                      int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream,
+                      int32_t q_len = 1, int32_t window = 0) {
     pa_status st;
     if (num_kv_heads != dims->num_kv_heads)
         return fail(PA_ERR_SHAPE, "num_kv_heads %d != dims->num_kv_heads %d", num_kv_heads, dims->num_kv_heads);
     Plan pl;
-    st = make_plan(dims, max_context_len, partition_tokens, &pl);
+    st = make_plan(dims, max_context_len, partition_tokens, &pl, q_len, window);
     if (st != PA_OK) return st;
     if (dims->num_seqs == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !context_lens || (!block_tables && dims->max_blocks_per_seq > 0))
@@ -141,12 +157,28 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
     p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.lse_off) : nullptr;
     const int g = dims->num_heads / dims->num_kv_heads;
+    p.group = g;
+    p.q_len = q_len;
+    p.window = window;
+    const int rows = row_capacity(g * q_len);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_fp8(dims);
-    cudaError_t e = !fp8 && pa::decode_tc_supported(dims->head_dim, g, dims->num_blocks, dims->num_kv_heads)
-                        ? pa::launch_decode_tc(p, dims->dtype, g, cs)
-                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, g, fp8, cs);
+    cudaError_t e = !fp8 && pa::decode_tc_supported(dims->head_dim, rows, dims->num_blocks, dims->num_kv_heads)
+                        ? pa::launch_decode_tc(p, dims->dtype, rows, cs)
+                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, rows, fp8, cs);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "pa_decode_fp8 launch" : "pa_decode launch");
+    return PA_OK;
+}
+
+pa_status check_opts(const pa_dims *d, const pa_decode_opts *o) {
+    if (!o) return fail(PA_ERR_NULL, "opts is NULL");
+    if (o->q_len < 1 || o->window < 0) return fail(PA_ERR_SHAPE, "q_len %d must be >= 1, window %d >= 0", o->q_len,
+                                                  o->window);
+    if (!(o->k_scale > 0.f) || !(o->v_scale > 0.f) || !isfinite(o->k_scale) || !isfinite(o->v_scale))
+        return fail(PA_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+    const int64_t rows = (int64_t)(d->num_heads / d->num_kv_heads) * o->q_len;
+    if (rows > 16) return fail(PA_ERR_UNSUPPORTED, "group * q_len = %lld: at most 16 query rows per KV head",
+                               (long long)rows);
     return PA_OK;
 }
 
@@ -201,6 +233,28 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
         return fail(PA_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
     return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale, num_kv_heads,
                        dims, max_context_len, partition_tokens, workspace, workspace_bytes, stream);
+}
+
+size_t pa_decode_ext_workspace_size(const pa_dims *dims, const pa_decode_opts *opts, int32_t max_context_len,
+                                    int32_t partition_tokens) {
+    if (check_dims(dims, true) != PA_OK || check_opts(dims, opts) != PA_OK) return (size_t)-1;
+    Plan pl;
+    if (make_plan(dims, max_context_len, partition_tokens, &pl, opts->q_len, opts->window) != PA_OK)
+        return (size_t)-1;
+    return pl.ws_bytes;
+}
+
+pa_status pa_decode_ext(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens, float scale, int32_t num_kv_heads,
+                        const pa_dims *dims, const pa_decode_opts *opts, int32_t max_context_len,
+                        int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream) {
+    pa_status st = check_dims(dims, true);
+    if (st != PA_OK) return st;
+    st = check_opts(dims, opts);
+    if (st != PA_OK) return st;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, opts->k_scale, opts->v_scale,
+                       num_kv_heads, dims, max_context_len, partition_tokens, workspace, workspace_bytes, stream,
+                       opts->q_len, opts->window);
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,

@@ -32,10 +32,6 @@ namespace {
 
 constexpr int kWarps = 4;
 
-__device__ __forceinline__ int part_lmax(const DecodeParams &p) {
-    return min(p.max_blocks_per_seq * kBlock, p.max_parts * p.part_blocks * kBlock);
-}
-
 // Shared-memory layout of the fixed-partition kernel (bytes):
 //   [main]  per-warp stage rings (kWarps x NSTAGE x {K chunk, V chunk}); reused
 //           at the end for the cross-warp reduction (kWarps x G x D floats)
@@ -60,7 +56,7 @@ struct PartLayout {
 // are half the bytes, so twice the stages keep as many bytes in flight.
 __host__ __device__ constexpr int part_stages(int G, int esz) { return (G <= 2 ? 2 : 3) * (esz == 1 ? 2 : 1); }
 
-template <typename T, typename KT, int D, int G, int NSTAGE>
+template <typename T, typename KT, int D, int G, int NSTAGE, bool kMasked>
 __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodeParams p) {
     constexpr int kEsz = std::is_same<KT, E4M3>::value ? 1 : 2;
     constexpr PartLayout S(D, G, NSTAGE, kEsz);
@@ -78,29 +74,47 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads;
-    const int head0 = kvh * G;
+    const int head0 = kvh * G;  // unmasked launches only (group == G, q_len == 1)
+    // flat q / out row of row r: plain decode keeps the group's rows contiguous
+    auto row_of = [&](int r) -> int64_t {
+        if constexpr (kMasked) return query_row(p, s, kvh, r);
+        return (int64_t)s * H + head0 + r;
+    };
+    const int rows = kMasked ? p.group * p.q_len : G;  // real rows (the rest is padding)
 
     pdl_launch_dependents();
     pdl_wait();
-    const int L = checked_len(p, s, part_lmax(p), part == 0 && kvh == 0 && tid == 0);
-    const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
+    const SeqSplit sp = seq_split(p, s, part == 0 && kvh == 0 && tid == 0);
+    const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part >= nparts) return;
     const bool direct = nparts == 1;
     T *out = reinterpret_cast<T *>(p.out);
 
     if (L == 0) {  // empty context: zero rows
-        for (int i = tid; i < G * D; i += blockDim.x)
-            out[((int64_t)s * H + head0 + i / D) * D + i % D] = E::from_float(0.f);
+        for (int i = tid; i < rows * D; i += blockDim.x) out[row_of(i / D) * D + i % D] = E::from_float(0.f);
         return;
     }
 
-    const int b0 = part * p.part_blocks;
+    int lo[G], hi[G];  // attended positions of each row (masked launches)
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+        if constexpr (kMasked) {
+            row_range(p, L, r, &lo[r], &hi[r]);
+        } else {
+            lo[r] = 0;
+            hi[r] = L - 1;
+        }
+    }
+
+    const int b0 = sp.bfirst + part * p.part_blocks;
     const int b1 = min(b0 + p.part_blocks, nblk);
     for (int i = tid; i < b1 - b0; i += blockDim.x)
         tbl[i] = (int32_t)checked_block(p, p.block_tables[(int64_t)s * p.max_blocks_per_seq + b0 + i]);
-    load_q_scaled<T, D, G>(q_s, reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * D, p.scale_log2, tid,
-                           blockDim.x);
+    if constexpr (kMasked)
+        load_q_rows_scaled<T, D, G>(q_s, p, s, kvh, tid, blockDim.x);
+    else
+        load_q_scaled<T, D, G>(q_s, reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * D, p.scale_log2,
+                               tid, blockDim.x);
     if (tid == 0) {
         fail_s = 0;
         for (int i = 0; i < kWarps * NSTAGE; ++i) mbar_init(&bars[i], 1);
@@ -139,7 +153,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
         }
         const unsigned char *ks = stages + st * 2 * S.chunk;
         const int base = (b0 + warp + kWarps * j) * kBlock;
-        simt_block<T, KT, D, G>(state, ks, ks + S.chunk, min(kBlock, L - base), q_s, pw, lane);
+        simt_block<T, KT, D, G, kMasked>(state, ks, ks + S.chunk, min(kBlock, L - base), q_s, pw, lane, base, lo, hi);
         if (lane == 0 && j + NSTAGE < nw) {
             fence_proxy_async_smem();
             issue(j + NSTAGE);
@@ -168,51 +182,55 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
         }
     }
     __syncthreads();
-    for (int i = tid; i < G * D; i += blockDim.x) {
+    for (int i = tid; i < rows * D; i += blockDim.x) {
         const int h = i / D, d = i % D;
         float lse;
         float o = combine_warps<D, G, kWarps>(red_m, red_l, red_acc, h, d, &lse);
-        if constexpr (kEsz == 1) o *= p.v_scale;  // FP8: V codes were unscaled
-        const int head = head0 + h;
+        o *= p.v_scale;  // V elements are read unscaled (v_scale = 1 for a plain 16-bit call)
+        const int64_t qr = row_of(h);
         if (direct) {
-            out[((int64_t)s * H + head) * D + d] = E::from_float(o);
+            out[qr * D + d] = E::from_float(o);
         } else {
-            const int64_t row = ((int64_t)s * H + head) * p.max_parts + part;
+            const int64_t row = qr * p.max_parts + part;
             p.ws_o[row * D + d] = o;
             if (d == 0) p.ws_lse[row] = lse;
         }
     }
 }
 
-// out[s, h, :] = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p,
-// over the partitions sequence s actually uses.  One CTA of D threads per (h, s).
+// out[row, :] = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p,
+// over the partitions sequence s actually uses (all -inf: a masked row with
+// no position, zero).  One CTA of D threads per (query token x head, s).
 template <typename T, int D>
 __global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p) {
-    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+    const int s = blockIdx.y, d = threadIdx.x;
     pdl_launch_dependents();
     pdl_wait();
-    const int L = checked_len(p, s, part_lmax(p), false);
-    const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
+    const SeqSplit sp = seq_split(p, s, false);
+    const int nparts = sp.nparts;
     if (nparts <= 1) return;  // written directly by the decode kernel
-    const int64_t row = ((int64_t)s * p.num_heads + h) * p.max_parts;
+    const int64_t qr = (int64_t)s * p.q_len * p.num_heads + blockIdx.x;
+    const int64_t row = qr * p.max_parts;
     const float *lse = p.ws_lse + row;
     float M = -INFINITY;
     for (int i = 0; i < nparts; ++i) M = fmaxf(M, lse[i]);
     float wsum = 0.f, o = 0.f;
-    for (int i = 0; i < nparts; ++i) {
-        const float w = exp2f(lse[i] - M);
-        wsum += w;
-        o = fmaf(w, p.ws_o[(row + i) * D + d], o);
+    if (M != -INFINITY) {
+        for (int i = 0; i < nparts; ++i) {
+            const float w = exp2f(lse[i] - M);
+            wsum += w;
+            o = fmaf(w, p.ws_o[(row + i) * D + d], o);
+        }
+        o /= wsum;
     }
-    reinterpret_cast<T *>(p.out)[((int64_t)s * p.num_heads + h) * D + d] = Elem<T>::from_float(o / wsum);
+    reinterpret_cast<T *>(p.out)[qr * D + d] = Elem<T>::from_float(o);
 }
 
-template <typename T, typename KT, int D, int G>
-cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
+template <typename T, typename KT, int D, int G, bool kMasked>
+cudaError_t launch_part_m(const DecodeParams &p, cudaStream_t stream) {
     constexpr int kEsz = std::is_same<KT, E4M3>::value ? 1 : 2;
     constexpr int kStages = part_stages(G, kEsz);
-    auto kern = decode_part_kernel<T, KT, D, G, kStages>;
+    auto kern = decode_part_kernel<T, KT, D, G, kStages, kMasked>;
     const int smem = PartLayout(D, G, kStages, kEsz).bytes(p.part_blocks);
     static int configured[kMaxDevices] = {};
     cudaError_t e = ensure_smem(kern, smem, configured);
@@ -220,6 +238,12 @@ cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
     e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(kWarps * 32), smem, stream, p);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, D, stream);
+}
+
+template <typename T, typename KT, int D, int G>
+cudaError_t launch_part_t(const DecodeParams &p, cudaStream_t stream) {
+    return decode_masked(p) ? launch_part_m<T, KT, D, G, true>(p, stream)
+                            : launch_part_m<T, KT, D, G, false>(p, stream);
 }
 
 template <typename T, typename KT, int D>
@@ -242,7 +266,7 @@ cudaError_t launch_part_k(const DecodeParams &p, int head_dim, int group, cudaSt
 }  // namespace
 
 cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream) {
-    const dim3 grid(p.num_heads, p.num_seqs);
+    const dim3 grid(p.num_heads * p.q_len, p.num_seqs);
     if (dtype == PA_F16)
         return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, dim3(64), 0, stream, p)
                               : launch_pdl(merge_part_kernel<__half, 128>, grid, dim3(128), 0, stream, p);
@@ -250,13 +274,13 @@ cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_d
                           : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p);
 }
 
-cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group, bool fp8_cache,
+cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int rows, bool fp8_cache,
                                       cudaStream_t stream) {
     if (dtype == PA_F16)
-        return fp8_cache ? launch_part_k<__half, E4M3>(p, head_dim, group, stream)
-                         : launch_part_k<__half, __half>(p, head_dim, group, stream);
-    return fp8_cache ? launch_part_k<__nv_bfloat16, E4M3>(p, head_dim, group, stream)
-                     : launch_part_k<__nv_bfloat16, __nv_bfloat16>(p, head_dim, group, stream);
+        return fp8_cache ? launch_part_k<__half, E4M3>(p, head_dim, rows, stream)
+                         : launch_part_k<__half, __half>(p, head_dim, rows, stream);
+    return fp8_cache ? launch_part_k<__nv_bfloat16, E4M3>(p, head_dim, rows, stream)
+                     : launch_part_k<__nv_bfloat16, __nv_bfloat16>(p, head_dim, rows, stream);
 }
 
 }  // namespace pa

@@ -27,7 +27,14 @@ struct DecodeParams {
     int64_t num_blocks;
     int32_t part_blocks;         // table entries per KV partition
     int32_t max_parts;           // partitions in the grid (gridDim.x)
+    int32_t group;               // query heads per KV head
+    int32_t q_len;               // query tokens per sequence (q, out: [S, q_len, H, D])
+    int32_t window;              // sliding window in tokens, 0 = none
 };
+
+// Whether a launch needs per-row position masks (several query tokens or a
+// sliding window); the kernels take this as a template flag.
+inline bool decode_masked(const DecodeParams &p) { return p.q_len != 1 || p.window != 0; }
 
 // Raise a kernel's dynamic shared-memory limit on the current device when a
 // launch needs more than was set before (the attribute is per device).
@@ -50,17 +57,18 @@ pa_status set_last_error(pa_status st, const char *msg);
 
 // Fixed-partition decode (+ merge when max_parts > 1) on `stream`; the
 // caches hold elements of `dtype`, or FP8 E4M3 codes when `fp8_cache`.
-cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int group, bool fp8_cache,
+// `rows` is the row capacity per KV head (1, 2, 4, 8 or 16 >= group * q_len).
+cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int rows, bool fp8_cache,
                                       cudaStream_t stream);
 
 
 // Log-sum-exp merge of the partitions written to the workspace.
 cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream);
 
-// Tensor-core decode for GQA groups (head_dim 128, group 4, 8 or 16) and
-// whether it applies to these sizes.
-bool decode_tc_supported(int head_dim, int group, int64_t num_blocks, int num_kv_heads);
-cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int group, cudaStream_t stream);
+// Tensor-core decode for row capacities 4, 8 or 16 at head_dim 128 (GQA
+// groups, or several query tokens) and whether it applies to these sizes.
+bool decode_tc_supported(int head_dim, int rows, int64_t num_blocks, int num_kv_heads);
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, cudaStream_t stream);
 
 // Cache kernels.
 struct CacheDims {

@@ -65,10 +65,6 @@ constexpr uint32_t kTmemCols = 64;
 __device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * kN); }
 __device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)(2 * kN + b * kN); }
 
-__device__ __forceinline__ int part_lmax_tc(const DecodeParams &p) {
-    return min(p.max_blocks_per_seq * kBlock, p.max_parts * p.part_blocks * kBlock);
-}
-
 __device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
 
 // Bounded wait that gives up at once when another thread already failed.
@@ -125,7 +121,9 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
 // groups of 16, whose per-thread state needs the registers of 2.
 __host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; }
 
-template <typename T, int G>
+// G: columns of S (query rows per KV head: the group, or group x query
+// tokens with kMasked, padded to a power of two).
+template <typename T, int G, bool kMasked>
 __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
@@ -147,19 +145,22 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
 
     const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.num_heads, head0 = kvh * G;
+    const int H = p.num_heads, head0 = kvh * G;  // head0: unmasked launches (group == G, q_len == 1)
     T *out = reinterpret_cast<T *>(p.out);
+    auto row_of = [&](int r) -> int64_t {
+        if constexpr (kMasked) return query_row(p, s, kvh, r);
+        return (int64_t)s * H + head0 + r;
+    };
+    const int rows = kMasked ? p.group * p.q_len : G;
 
     pdl_launch_dependents();
     pdl_wait();
-    const int L = checked_len(p, s, part_lmax_tc(p), part == 0 && kvh == 0 && tid == 0);
-    const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
+    const SeqSplit sp = seq_split(p, s, part == 0 && kvh == 0 && tid == 0);
+    const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part >= nparts) return;
     const bool direct = nparts == 1;
     if (L == 0) {
-        for (int i = tid; i < G * kD; i += blockDim.x)
-            out[((int64_t)s * H + head0 + i / kD) * kD + i % kD] = E::from_float(0.f);
+        for (int i = tid; i < rows * kD; i += blockDim.x) out[row_of(i / kD) * kD + i % kD] = E::from_float(0.f);
         return;
     }
     // The swizzled tiles need a 1024-byte aligned base; never touch them otherwise.
@@ -167,7 +168,7 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
         if (tid == 0) flag_error(PA_DEVERR_LAYOUT);
         return;
     }
-    const int b0 = part * p.part_blocks;
+    const int b0 = sp.bfirst + part * p.part_blocks;
     const int nb = min(p.part_blocks, nblk - b0);          // blocks of this partition
     const int nch = (nb + kChunkBlocks - 1) / kChunkBlocks; // chunks of 128 tokens
     const int tok0 = b0 * kBlock;
@@ -245,11 +246,11 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
             // Q tile: rows = the group's query heads (zero rows up to 16),
             // K-major 128-byte swizzle, two 64-dim regions.  Loaded while the
             // producers already stream K and V.
-            const T *q = reinterpret_cast<const T *>(p.q) + ((int64_t)s * H + head0) * kD;
+            const T *q = reinterpret_cast<const T *>(p.q);
             for (int i = tid; i < kN * (kD / 8); i += 128) {
                 const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
                 uint4 v = make_uint4(0, 0, 0, 0);
-                if (r < G) v = *reinterpret_cast<const uint4 *>(q + r * kD + c16 * 8);
+                if (r < rows) v = *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + c16 * 8);
                 *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
             }
             fence_proxy_async_smem();
@@ -257,6 +258,16 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
         }
         const int t = tid;                                      // token of S, dim of O
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // TMEM lane quadrant
+        int lo[G], hi[G];  // attended positions of each column (masked launches)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            if constexpr (kMasked) {
+                row_range(p, L, h, &lo[h], &hi[h]);
+            } else {
+                lo[h] = 0;
+                hi[h] = L - 1;
+            }
+        }
         float m[G], l[G], acc[G], alpha_prev[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -286,7 +297,9 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
                 tc::tmem_ld<kCols>(tmem + lane_base + s_col(c & 1), sv);
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    x[h] = valid ? sv[h] * p.scale_log2 : -INFINITY;
+                    bool live = valid;
+                    if constexpr (kMasked) live = live && tok >= lo[h] && tok <= hi[h];
+                    x[h] = live ? sv[h] * p.scale_log2 : -INFINITY;
                     exceed |= x[h] > m[h] + kLazyMax;
                 }
             } else {
@@ -326,7 +339,8 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
             T pv[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                pv[h] = E::from_float(ex2(x[h] - m[h]));
+                // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
+                pv[h] = (kMasked && x[h] == -INFINITY) ? E::from_float(0.f) : E::from_float(ex2(x[h] - m[h]));
                 l[h] += E::to_float(pv[h]);  // the rounded weight the MMA sees
             }
             if (c > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
@@ -372,13 +386,27 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 const float lt = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
-                const float o = acc[h] / lt;
-                if (direct) {
-                    out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
-                } else {
-                    const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
-                    p.ws_o[r * kD + t] = o;
-                    if (t == 0) p.ws_lse[r] = m[h] + log2f(lt);
+                if constexpr (kMasked) {
+                    if (h >= rows) break;
+                    // lt = 0 only for a column with no position in this partition
+                    const float o = lt > 0.f ? acc[h] / lt * p.v_scale : 0.f;
+                    const int64_t qr = row_of(h);
+                    if (direct) {
+                        out[qr * kD + t] = E::from_float(o);
+                    } else {
+                        const int64_t r = qr * p.max_parts + part;
+                        p.ws_o[r * kD + t] = o;
+                        if (t == 0) p.ws_lse[r] = lt > 0.f ? m[h] + log2f(lt) : -INFINITY;
+                    }
+                } else {  // plain decode: every column has tokens, V unscaled
+                    const float o = acc[h] / lt;
+                    if (direct) {
+                        out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
+                    } else {
+                        const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
+                        p.ws_o[r * kD + t] = o;
+                        if (t == 0) p.ws_lse[r] = m[h] + log2f(lt);
+                    }
                 }
             }
         }
@@ -425,14 +453,14 @@ bool encode_cache_map(CUtensorMap *map, const void *base, int64_t rows, bool bf1
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int G>
+template <typename T, int G, bool kMasked>
 cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
     CUtensorMap tk, tv;
     if (!encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) ||
         !encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value))
         return cudaErrorInvalidValue;
-    auto kern = decode_tc_kernel<T, G>;
+    auto kern = decode_tc_kernel<T, G, kMasked>;
     static int configured[kMaxDevices] = {};
     static int carveout_set[kMaxDevices] = {};
     int dev = 0;
@@ -451,25 +479,33 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
 }
 
-template <typename T>
-cudaError_t launch_tc_d(const DecodeParams &p, int group, cudaStream_t stream) {
-    switch (group) {
-        case 4: return launch_tc_t<T, 4>(p, stream);
-        case 8: return launch_tc_t<T, 8>(p, stream);
-        case 16: return launch_tc_t<T, 16>(p, stream);
+template <typename T, bool kMasked>
+cudaError_t launch_tc_m(const DecodeParams &p, int rows, cudaStream_t stream) {
+    switch (rows) {
+        case 4: return launch_tc_t<T, 4, kMasked>(p, stream);
+        case 8: return launch_tc_t<T, 8, kMasked>(p, stream);
+        case 16: return launch_tc_t<T, 16, kMasked>(p, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
+// The plain variant neither masks nor scales V: anything else takes the
+// masked one (with q_len = 1, no window its masks keep every token).
+template <typename T>
+cudaError_t launch_tc_d(const DecodeParams &p, int rows, cudaStream_t stream) {
+    return decode_masked(p) || p.v_scale != 1.f ? launch_tc_m<T, true>(p, rows, stream)
+                                                : launch_tc_m<T, false>(p, rows, stream);
+}
+
 }  // namespace
 
-bool decode_tc_supported(int head_dim, int group, int64_t num_blocks, int num_kv_heads) {
-    return head_dim == kD && (group == 4 || group == 8 || group == 16) &&
+bool decode_tc_supported(int head_dim, int rows, int64_t num_blocks, int num_kv_heads) {
+    return head_dim == kD && (rows == 4 || rows == 8 || rows == 16) &&
            num_blocks * num_kv_heads * kBlock < ((int64_t)1 << 31) - kBlock;
 }
 
-cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int group, cudaStream_t stream) {
-    return dtype == PA_F16 ? launch_tc_d<__half>(p, group, stream) : launch_tc_d<__nv_bfloat16>(p, group, stream);
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, cudaStream_t stream) {
+    return dtype == PA_F16 ? launch_tc_d<__half>(p, rows, stream) : launch_tc_d<__nv_bfloat16>(p, rows, stream);
 }
 
 }  // namespace pa

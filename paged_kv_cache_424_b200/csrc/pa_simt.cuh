@@ -46,6 +46,50 @@ __device__ __forceinline__ int64_t checked_block(const DecodeParams &p, int32_t 
     return b;
 }
 
+// First table entry any query of a sequence of L tokens reads: 0, or with a
+// sliding window the block holding the earliest attended position (that of
+// query token 0, L - q_len - window + 1).
+__device__ __forceinline__ int first_block(const DecodeParams &p, int L) {
+    if (p.window <= 0) return 0;
+    const int lo = L - p.q_len - p.window + 1;
+    return lo > 0 ? lo / kBlock : 0;
+}
+
+// How sequence s is split: its checked length, its first block, its blocks
+// and its partitions (table entries [bfirst + i * part_blocks, ...) for
+// partition i).  Every decode kernel and the merge use this one rule.
+struct SeqSplit {
+    int L, bfirst, nblk, nparts;
+};
+__device__ __forceinline__ SeqSplit seq_split(const DecodeParams &p, int s, bool report) {
+    SeqSplit r;
+    const bool masked = p.q_len != 1 || p.window != 0;
+    const int lmax_table = p.max_blocks_per_seq * kBlock;
+    r.L = checked_len(p, s, masked ? lmax_table : min(lmax_table, p.max_parts * p.part_blocks * kBlock), report);
+    r.nblk = (r.L + kBlock - 1) / kBlock;
+    r.bfirst = first_block(p, r.L);
+    r.nparts = r.nblk == 0 ? 1 : (r.nblk - r.bfirst + p.part_blocks - 1) / p.part_blocks;
+    if (r.nparts > p.max_parts) {  // longer than the plan's max_context_len: flagged, cut
+        if (report) flag_error(PA_DEVERR_CONTEXT);
+        r.nparts = p.max_parts;
+    }
+    return r;
+}
+
+// Flat index of query row r of KV head kvh of sequence s in q / out ([S,
+// q_len, H] rows): query token r / group, head kvh * group + r % group.
+__device__ __forceinline__ int64_t query_row(const DecodeParams &p, int s, int kvh, int r) {
+    return ((int64_t)s * p.q_len + r / p.group) * p.num_heads + kvh * p.group + r % p.group;
+}
+
+// Attended positions [lo, hi] of query row r of a sequence of L tokens
+// (hi < 0: none; rows past group * q_len are padding and attend nothing).
+__device__ __forceinline__ void row_range(const DecodeParams &p, int L, int r, int *lo, int *hi) {
+    const int h = r < p.group * p.q_len ? L - p.q_len + r / p.group : -1;
+    *hi = h;
+    *lo = p.window > 0 && h - p.window + 1 > 0 ? h - p.window + 1 : 0;
+}
+
 // Query rows of a KV-head group in shared memory: fp32, pre-scaled into the
 // log2 domain, laid out [h][half][chunk][12] (8 used + 4 pad floats per
 // 8-element chunk) so the rotated chunk reads of simt_block are free of
@@ -67,6 +111,24 @@ __device__ __forceinline__ void load_q_scaled(float *q_s, const T *q_rows, float
         float *dst = q_s + (h * 2 + half) * SimtQ<D>::kHalf + (e / 8) * 12 + (e % 8);
         dst[0] = f.x * scale_log2;
         dst[1] = f.y * scale_log2;
+    }
+}
+
+// The same for rows spread over several query tokens: row r is
+// q[query_row(p, s, kvh, r)]; padding rows (r >= group * q_len) are zero.
+template <typename T, int D, int G>
+__device__ __forceinline__ void load_q_rows_scaled(float *q_s, const DecodeParams &p, int s, int kvh, int tid,
+                                                   int nthreads) {
+    const T *q = reinterpret_cast<const T *>(p.q);
+    const int rows = p.group * p.q_len;
+    for (int i = tid; i < G * D / 2; i += nthreads) {
+        const int h = i / (D / 2), e2 = (i % (D / 2)) * 2;
+        float2 f = make_float2(0.f, 0.f);
+        if (h < rows) f = Elem<T>::to_float2(*reinterpret_cast<const uint32_t *>(q + query_row(p, s, kvh, h) * D + e2));
+        const int half = e2 / (D / 2), e = e2 % (D / 2);
+        float *dst = q_s + (h * 2 + half) * SimtQ<D>::kHalf + (e / 8) * 12 + (e % 8);
+        dst[0] = f.x * p.scale_log2;
+        dst[1] = f.y * p.scale_log2;
     }
 }
 
@@ -110,9 +172,12 @@ __device__ __forceinline__ float ex2(float x) {
 // memory, elements of KT (T itself, or E4M3 codes whose scale the caller
 // folds into q and the output); pw: this warp's G x 16 float scratch for the
 // softmax weights.
-template <typename T, typename KT, int D, int G>
+// With kMasked, row h sees only positions lo[h] .. hi[h]; `base` is the
+// block's first position.
+template <typename T, typename KT, int D, int G, bool kMasked = false>
 __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned char *ks, const unsigned char *vs,
-                                           int nvalid, const float *q_s, float *pw, int lane) {
+                                           int nvalid, const float *q_s, float *pw, int lane, int base = 0,
+                                           const int *lo = nullptr, const int *hi = nullptr) {
     using E = Elem<T>;
     constexpr bool kFp8 = std::is_same<KT, E4M3>::value;
     constexpr int kEsz = kFp8 ? 1 : 2;   // bytes per cache element
@@ -185,7 +250,9 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
 #pragma unroll
         for (int a = 1; a < NA; ++a) v += x[h][a];
         v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v = (t < nvalid) ? v : -INFINITY;
+        bool live = t < nvalid;
+        if constexpr (kMasked) live = live && base + t >= lo[h] && base + t <= hi[h];
+        v = live ? v : -INFINITY;
         if (__any_sync(0xffffffffu, v > st.m[h] + kLazyMax)) {
             // rare: raise the running max to this block's max and rescale
             float bm = v;
@@ -200,7 +267,8 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
             for (int e = 0; e < kPV; ++e) st.acc[h][e] *= alpha;
             st.m[h] = mn;
         }
-        const float pr = ex2(v - st.m[h]);
+        // masked rows may still have m = -inf: their weight is 0, not 2^(-inf + inf)
+        const float pr = (kMasked && v == -INFINITY) ? 0.f : ex2(v - st.m[h]);
         if (half == 0) {
             st.l[h] += pr;
             pw[h * kBlock + t] = pr;
@@ -274,13 +342,18 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
 // Cross-warp combination of NW warp states stored as red_m/red_l [NW][G] and
 // red_acc [NW][G][D]: for element (h, d) returns o = sum_w 2^(m_w - M) acc_w /
 // sum_w 2^(m_w - M) l_w and lse = M + log2(sum_w 2^(m_w - M) l_w).  Warps
-// that saw no block have m = -inf and l = acc = 0 and drop out.
+// that saw no block have m = -inf and l = acc = 0 and drop out; a row that
+// no warp saw (possible only with masks) gives o = 0, lse = -inf.
 template <int D, int G, int NW>
 __device__ __forceinline__ float combine_warps(const float *red_m, const float *red_l, const float *red_acc, int h,
                                                int d, float *lse) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * G + h]);
+    if (M == -INFINITY) {  // a masked row with no position in this partition
+        *lse = -INFINITY;
+        return 0.f;
+    }
     float lsum = 0.f, o = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {

@@ -122,6 +122,8 @@ class DeviceSession:
         inp = inputs or self.decode_inputs(step)
         P = self.sc.partition_tokens if partition_tokens is None else partition_tokens
         maxlen = step.max_context_len
+        if self.sc.ext:
+            return self.decode_ext(inp, maxlen, P, out)
         dims = pa.dims_of(inp["q"], self.k_cache, inp["block_tables"])
         ws = self.workspace(pa.pa_decode_workspace_size(dims, maxlen, P))
         if out is None:
@@ -132,6 +134,29 @@ class DeviceSession:
         else:
             pa.pa_decode(out, inp["q"], self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"],
                          self.sc.scale, d.num_kv_heads, maxlen, P, ws)
+        return out
+
+    def ext_workspace_bytes(self, inp: Dict[str, torch.Tensor], maxlen: int, P: int) -> int:
+        sc = self.sc
+        q4 = inp["q"] if inp["q"].dim() == 4 else inp["q"][:, None]
+        dims = pa.ext_dims(q4, self.k_cache, inp["block_tables"])
+        opts = pa.pa_decode_opts(sc.q_len, sc.window, sc.k_scale, sc.v_scale)
+        return pa.pa_decode_ext_workspace_size(dims, opts, maxlen, P)
+
+    def decode_ext(self, inp: Dict[str, torch.Tensor], maxlen: int, P: int,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Multi-token / sliding-window decode of the scenario (q [S, q_len,
+        H, D], or [S, H, D] for one token with a window)."""
+        sc = self.sc
+        q = inp["q"]
+        q4 = q if q.dim() == 4 else q[:, None]
+        ws = self.workspace(self.ext_workspace_bytes(inp, maxlen, P))
+        if out is None:
+            out = torch.empty_like(q)
+        out4 = out if out.dim() == 4 else out[:, None]
+        pa.pa_decode_ext(out4, q4, self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"], sc.scale,
+                         sc.dims.num_kv_heads, maxlen, sc.q_len, sc.window, sc.k_scale, sc.v_scale, P, ws,
+                         stream=stream)
         return out
 
     def run_step(self, step: Step, partition_tokens: Optional[int] = None) -> torch.Tensor:

@@ -141,6 +141,16 @@ class Scenario:
     kv_dtype: str = ""
     k_scale: float = 1.0
     v_scale: float = 1.0
+    # Multi-token / sliding-window decode: each step writes q_len new tokens
+    # per sequence and queries all of them (q is [S, q_len, H, D] when
+    # q_len > 1); window > 0 limits every query to its `window` most recent
+    # positions.
+    q_len: int = 1
+    window: int = 0
+
+    @property
+    def ext(self) -> bool:
+        return self.q_len != 1 or self.window != 0
 
     @property
     def kv_elem_bytes(self) -> int:
@@ -202,31 +212,41 @@ class _Builder:
     def new_sequence(self, length: int) -> Tuple[SeqBlocks, int]:
         """A sequence whose first ``length - 1`` tokens are prefilled; returns
         it and the slot of its last token, which the step's write fills."""
+        seq, slots = self.new_sequence_multi(length, 1)
+        return seq, slots[0]
+
+    def new_sequence_multi(self, length: int, new: int) -> Tuple[SeqBlocks, List[int]]:
+        """A sequence whose first ``length - new`` tokens are prefilled (at
+        least none); returns it and the slots of its last ``new`` tokens,
+        which the step's write fills."""
         seq = self.bm.new_sequence()
-        for _ in range(length - 1):
+        pre = max(0, length - new)
+        for _ in range(pre):
             self.bm.append_slot(seq)
-        self.fill(seq.blocks, length - 1)
-        slot = self.bm.append_slot(seq)
-        if len(seq.blocks) > (length - 1 + self.dims.block_size - 1) // self.dims.block_size:
-            # the decode token opened a new block: admit it as all-NaN
-            self.fill(seq.blocks[-1:], 0)
-        return seq, slot
+        self.fill(seq.blocks, pre)
+        before = len(seq.blocks)
+        slots = [self.bm.append_slot(seq) for _ in range(length - pre)]
+        if len(seq.blocks) > before:
+            # the new tokens opened blocks: admit them as all-NaN
+            self.fill(seq.blocks[before:], 0)
+        return seq, slots
 
     def new_tokens(self, n: int) -> Tuple[np.ndarray, np.ndarray]:
         d = self.dims
         shape = (n, d.num_kv_heads, d.head_dim)
         return uniform_bits(self.rng, shape, d.dtype), uniform_bits(self.rng, shape, d.dtype, lo=self.v_lo)
 
-    def queries(self) -> np.ndarray:
+    def queries(self, q_len: int = 1) -> np.ndarray:
         d = self.dims
-        return uniform_bits(self.rng, (d.num_seqs, d.num_heads, d.head_dim), d.dtype)
+        shape = (d.num_seqs, d.num_heads, d.head_dim) if q_len == 1 else (d.num_seqs, q_len, d.num_heads, d.head_dim)
+        return uniform_bits(self.rng, shape, d.dtype)
 
-    def step(self, seqs: List[SeqBlocks], writes: List[Write]) -> Step:
+    def step(self, seqs: List[SeqBlocks], writes: List[Write], q_len: int = 1) -> Step:
         d = self.dims
         ids, k, v = self.take_admitted()
         return Step(admit_ids=ids, admit_k=k, admit_v=v,
                     block_mapping=self.bm.take_copy_pairs(), writes=writes,
-                    q=self.queries(),
+                    q=self.queries(q_len),
                     block_tables=_tables(seqs, d.max_blocks_per_seq, self.pad_block),
                     context_lens=np.asarray([s.length for s in seqs], dtype=np.int32))
 
@@ -236,19 +256,22 @@ def _scale(head_dim: int) -> float:
 
 
 def _fresh_batch(name: str, dims: Dims, lengths: Sequence[int], rng: np.random.Generator,
-                 partition_tokens: int = 0, v_lo: float = -1.0, note: str = "") -> Scenario:
-    """One decode step over new sequences of the given lengths."""
+                 partition_tokens: int = 0, v_lo: float = -1.0, note: str = "", q_len: int = 1,
+                 window: int = 0) -> Scenario:
+    """One decode step over new sequences of the given lengths (the last
+    q_len tokens of each are the step's new tokens)."""
     b = _Builder(rng, dims, v_lo=v_lo)
     b.admit_pad()
     seqs, slots = [], []
     for L in lengths:
-        s, slot = b.new_sequence(int(L))
+        s, sl = b.new_sequence_multi(int(L), q_len)
         seqs.append(s)
-        slots.append(slot)
-    key, value = b.new_tokens(len(seqs))
+        slots.extend(sl)
+    key, value = b.new_tokens(len(slots))
     w = Write(key, value, np.asarray(slots, dtype=np.int64))
-    st = b.step(seqs, [w])
-    return Scenario(name, dims, _scale(dims.head_dim), b.pad_block, [st], partition_tokens, note)
+    st = b.step(seqs, [w], q_len)
+    return Scenario(name, dims, _scale(dims.head_dim), b.pad_block, [st], partition_tokens, note, q_len=q_len,
+                    window=window)
 
 
 # --------------------------------------------------------------------------
@@ -373,6 +396,35 @@ def cow(seed: int = 4, num_prompts: int = 16, samples: int = 8, prefix: int = 10
                     shared_blocks=np.asarray(shared, np.int64))
 
 
+def spec8b(seed: int = 5, num_seqs: int = 256, q_len: int = 4, median: int = 1024, cap: int = 4096,
+           num_blocks: int = 131072, window: int = 0, v_lo: float = -1.0) -> Scenario:
+    """Speculative verification on the 8B shape: every sequence of a
+    lognormal length mix (as gqa8b) writes q_len new tokens (the token being
+    decoded and q_len - 1 draft tokens) and queries all of them, each
+    causally; group 4 x 4 tokens fill the 16 query rows of a KV head."""
+    rng = np.random.default_rng(seed)
+    lengths = np.maximum(lognormal_lengths(rng, num_seqs, median, 1.0, cap), q_len)
+    mb = -(-cap // BLOCK_SIZE)
+    dims = Dims(num_seqs, 32, 8, 128, BLOCK_SIZE, mb, num_blocks, "bf16")
+    return _fresh_batch("spec8b", dims, lengths, rng, v_lo=v_lo, q_len=q_len, window=window,
+                        note=f"{num_seqs} seqs, lognormal(median {median}, sigma 1, cap {cap}), {q_len} query "
+                             f"tokens each, H=32/Hk=8, D=128, bf16, pool {num_blocks}")
+
+
+def window70b(seed: int = 6, num_seqs: int = 8, context_len: int = 32768, window: int = 4096,
+              num_blocks: int = 32768, q_len: int = 1, partition_tokens: int = 0, v_lo: float = -1.0) -> Scenario:
+    """The 70B long-context shape with a sliding window: each query attends
+    to its `window` most recent positions, so a step reads window tokens per
+    sequence whatever the context length."""
+    rng = np.random.default_rng(seed)
+    mb = -(-context_len // BLOCK_SIZE)
+    dims = Dims(num_seqs, 64, 8, 128, BLOCK_SIZE, mb, num_blocks, "bf16")
+    return _fresh_batch("window70b", dims, [context_len] * num_seqs, rng, partition_tokens, v_lo=v_lo,
+                        q_len=q_len, window=window,
+                        note=f"{num_seqs} seqs x {context_len} tokens, sliding window {window}, H=64/Hk=8, "
+                             f"D=128, bf16, pool {num_blocks}")
+
+
 # Per-tensor FP8 scales for inputs in [-1, 1]: |x| / scale reaches 81 (K)
 # and 141 (V), inside E4M3's range (448).  Not powers of two, so the
 # division before rounding is inexact and both sides must round it alike.
@@ -387,19 +439,31 @@ def with_fp8_cache(sc: Scenario, k_scale: float = FP8_K_SCALE, v_scale: float = 
                    note=f"{sc.note}; FP8 E4M3 cache, k_scale {k_scale}, v_scale {v_scale}")
 
 
-SCENARIOS = {"tiny": tiny, "mha7b": mha7b, "gqa8b": gqa8b, "long70b": long70b, "cow": cow}
+SCENARIOS = {"tiny": tiny, "mha7b": mha7b, "gqa8b": gqa8b, "long70b": long70b, "cow": cow, "spec8b": spec8b,
+             "window70b": window70b}
 CONFIG_ORDER = ["tiny", "mha7b", "gqa8b", "long70b", "cow"]
 
 
-def kv_bytes(step: Step, dims: Dims, unique: bool = False, elem_bytes: int = 2) -> int:
-    """KV bytes a decode step must read: sum of context lengths x 2 (K and V)
-    x KV heads x head_dim x element size (2 bytes; 1 for an FP8 cache).  With
-    ``unique``, blocks shared by several sequences count once (whole blocks,
-    partial tails as their token count)."""
+def attended_tokens(step: Step, q_len: int = 1, window: int = 0) -> np.ndarray:
+    """Per sequence, the positions some query attends to: all of them, or
+    with a window those from query 0's first (len - q_len - window + 1)."""
+    L = step.context_lens.astype(np.int64)
+    if window <= 0:
+        return L
+    return L - np.maximum(0, L - q_len - window + 1)
+
+
+def kv_bytes(step: Step, dims: Dims, unique: bool = False, elem_bytes: int = 2, q_len: int = 1,
+             window: int = 0) -> int:
+    """KV bytes a decode step must read: sum of attended tokens (the context
+    lengths, or the window spans) x 2 (K and V) x KV heads x head_dim x
+    element size (2 bytes; 1 for an FP8 cache).  With ``unique``, blocks
+    shared by several sequences count once (whole blocks, partial tails as
+    their token count)."""
     el = elem_bytes
     per_tok = 2 * dims.num_kv_heads * dims.head_dim * el
     if not unique:
-        return int(step.context_lens.astype(np.int64).sum()) * per_tok
+        return int(attended_tokens(step, q_len, window).sum()) * per_tok
     seen = {}
     for s in range(dims.num_seqs):
         L = int(step.context_lens[s])
@@ -411,6 +475,6 @@ def kv_bytes(step: Step, dims: Dims, unique: bool = False, elem_bytes: int = 2) 
     return sum(seen.values()) * per_tok
 
 
-def qo_bytes(dims: Dims) -> int:
-    """Query read + output write: 2 x S x H x D x 2 bytes."""
-    return 2 * dims.num_seqs * dims.num_heads * dims.head_dim * 2
+def qo_bytes(dims: Dims, q_len: int = 1) -> int:
+    """Query read + output write: 2 x S x q_len x H x D x 2 bytes."""
+    return 2 * dims.num_seqs * q_len * dims.num_heads * dims.head_dim * 2

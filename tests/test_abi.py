@@ -94,6 +94,24 @@ def test_fp8_cache_plans_on_the_cuda_core_kernel(lib):
     assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=lib.PA_BF16), 1024, 0) == 1
 
 
+def test_ext_plan_and_workspace(lib):
+    """Multi-token queries multiply the partial rows; a window bounds the
+    partitions by the attended span, not by the longest context."""
+    d = _dims(lib, num_heads=8)                      # group 1
+    O = lib.pa_decode_opts
+    plain = lib.pa_decode_workspace_size(d, 4096, 512)
+    assert lib.pa_decode_ext_workspace_size(d, O(1, 0, 1.0, 1.0), 4096, 512) == plain
+    ws4 = lib.pa_decode_ext_workspace_size(d, O(4, 0, 1.0, 1.0), 4096, 512)
+    rows4 = 4 * 4 * 8 * 8                            # S x q_len x H x partitions of 512
+    assert ws4 >= rows4 * 128 * 4 + rows4 * 4 and ws4 > plain
+    # window 1000 + 3 extra query tokens: at most ceil(1003 / 16) + 1 = 64 blocks -> 2 partitions of 512
+    wsw = lib.pa_decode_ext_workspace_size(d, O(4, 1000, 1.0, 1.0), 4096, 512)
+    rowsw = 4 * 4 * 8 * 2
+    assert rowsw * 128 * 4 <= wsw < ws4
+    assert lib.pa_decode_ext_workspace_size(d, O(1, 100, 1.0, 1.0), 4096, 512) == 0  # one partition
+    assert lib.LIB.pa_decode_ext_workspace_size(ctypes.byref(d), None, 100, 0) == ctypes.c_size_t(-1).value
+
+
 def test_bad_partition_and_context(lib):
     d = _dims(lib)
     assert lib.LIB.pa_decode_num_partitions(ctypes.byref(d), 100, 24) == -3   # not a multiple of 16
@@ -173,6 +191,22 @@ assert rc8(f8, n=-1) == -3
 assert rc8(f8, key=None) == -1
 assert rc8(f8, key=ctypes.c_void_p(0x10004)) == -7
 assert rc8(f8, key=None, n=0) == 0
+
+# pa_decode_ext: options are checked before anything else
+def ext(d, opts, ptrs=good, maxlen=100, ws=None, wsb=0):
+    out, q, k, v, bt, cl = ptrs
+    return L.pa_decode_ext(out, q, k, v, bt, cl, ctypes.c_float(0.1), 8, ctypes.byref(d),
+                           ctypes.byref(opts) if opts is not None else None, maxlen, 0, ws, wsb, None)
+O = lib.pa_decode_opts
+assert ext(d, None) == -1
+assert ext(d, O(0, 0, 1.0, 1.0)) == -3                 # q_len < 1
+assert ext(d, O(1, -1, 1.0, 1.0)) == -3                # window < 0
+assert ext(d, O(1, 0, 0.0, 1.0)) == -3                 # scale
+assert ext(d, O(1, 0, 1.0, float("nan"))) == -3
+assert ext(d, O(5, 0, 1.0, 1.0)) == -4                 # group 4 x 5 query tokens > 16
+assert ext(d, O(4, 0, 1.0, 1.0), ptrs=[None] + good[1:]) == -1
+assert ext(d, O(4, 0, 1.0, 1.0), maxlen=2000) == -5    # split, no workspace
+assert ext(dims(num_seqs=0), O(2, 64, 1.0, 1.0), ptrs=[None] * 6) == 0
 print("host checks ok")
 """
 
