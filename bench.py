@@ -49,14 +49,17 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha7b",
-                    choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "spec8b", "window70b", "swap"],
+                    choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "spec8b", "window70b", "prefix8b", "swap"],
                     help="decode scenario (spec8b: 4 query tokens per sequence; window70b: 4096-token sliding "
-                         "window), or 'swap' for pa_swap_blocks device <-> pinned host throughput")
+                         "window; prefix8b: shuffled batch of shared 2000-token prefixes, decoded in "
+                         "shared-prefix order), or 'swap' for pa_swap_blocks device <-> pinned host throughput")
     ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
     ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
     ap.add_argument("--kv", choices=["16", "fp8"], default="16",
                     help="KV cache element type: the 16-bit dtype of the workload, or FP8 E4M3 with scales")
+    ap.add_argument("--no-prefix-order", action="store_true",
+                    help="prefix8b: decode in plain batch order (no seq_order), for profiling the difference")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
@@ -78,10 +81,10 @@ def _base_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
         kw["num_blocks"] = num_blocks
     if name == "tiny":
         return W.tiny(seed)
-    if name == "cow":
+    if name in ("cow", "prefix8b"):
         if num_seqs is not None:
             kw = {"num_prompts": max(1, num_seqs // 8), **({"num_blocks": num_blocks} if num_blocks else {})}
-        return W.cow(seed, **kw)
+        return getattr(W, name)(seed, **kw)
     return getattr(W, name)(seed, **kw)
 
 
@@ -252,6 +255,9 @@ def run_ours(args):
     from paged_kv_cache_424_b200.session import DeviceSession, to_device
 
     sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv)
+    if args.no_prefix_order and sc.prefix_order:
+        import dataclasses
+        sc = dataclasses.replace(sc, prefix_order=False)
     st = sc.steps[0]
     d = sc.dims
     fp8 = sc.kv_dtype == "fp8"
@@ -262,11 +268,11 @@ def run_ours(args):
     writes = dev.write_inputs(st)
     bm = torch.from_numpy(np.ascontiguousarray(st.block_mapping)).to(device) if st.block_mapping.size else None
     maxlen = st.max_context_len
-    dims = pa.dims_of(inp["q"], dev.k_cache, inp["block_tables"])
     if sc.ext:
         ws_bytes = dev.ext_workspace_bytes(inp, maxlen, P)
         nparts = "split" if ws_bytes else 1
     else:
+        dims = pa.dims_of(inp["q"], dev.k_cache, inp["block_tables"])
         nparts = pa.pa_decode_num_partitions(dims, maxlen, P)
         ws_bytes = pa.pa_decode_workspace_size(dims, maxlen, P)
     ws = dev.workspace(ws_bytes)
@@ -280,9 +286,10 @@ def run_ours(args):
         else:
             pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
 
-    def decode(q, bt, cl):
+    def decode(q, bt, cl, seq_order=None):
         if sc.ext:
-            dev.decode_ext({"q": q, "block_tables": bt, "context_lens": cl}, maxlen, P, out, stream=stream)
+            dev.decode_ext({"q": q, "block_tables": bt, "context_lens": cl, "seq_order": seq_order}, maxlen, P, out,
+                           stream=stream)
         elif fp8:
             pa.pa_decode_fp8(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.k_scale, sc.v_scale,
                              d.num_kv_heads, maxlen, P, ws, stream=stream)
@@ -297,7 +304,7 @@ def run_ours(args):
             write(key, value, slots)
         if e0 is not None:
             e0.record(stream)
-        decode(inp["q"], inp["block_tables"], inp["context_lens"])
+        decode(inp["q"], inp["block_tables"], inp["context_lens"], inp.get("seq_order"))
         if e1 is not None:
             e1.record(stream)
 
@@ -326,6 +333,21 @@ def run_ours(args):
     dec_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
     dec_avg_ms = max_over_ranks(sum(dec_ms) / K, world, device)
 
+    # shared-prefix order: the same decode in plain batch order, for comparison
+    no_order_ms = None
+    if sc.prefix_order:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            decode(inp["q"], inp["block_tables"], inp["context_lens"], None)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        for _ in range(K):
+            decode(inp["q"], inp["block_tables"], inp["context_lens"], None)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        no_order_ms = max_over_ranks(a.elapsed_time(b) / K, world, device)
+
     # ---- end to end: host buffers in, result out, through the same calls ----
     e2e = None
     if not args.no_e2e:
@@ -340,7 +362,10 @@ def run_ours(args):
         d_w = [(torch.empty_like(k), torch.empty_like(v), torch.empty_like(s)) for k, v, s in writes]
         h_bm_t = torch.from_numpy(np.ascontiguousarray(h_bm)).pin_memory() if bm is not None else None
         d_bm = torch.empty_like(bm) if bm is not None else None
-        h2d = (h_q.numel() * h_q.element_size() + h_bt.numel() * 4 + h_cl.numel() * 4 +
+        d_so = torch.empty(d.num_seqs, dtype=torch.int32, device=device) if sc.prefix_order else None
+        h_so = torch.empty(d.num_seqs, dtype=torch.int32).pin_memory() if sc.prefix_order else None
+        h2d = ((h_so.numel() * 4 if h_so is not None else 0) +
+               h_q.numel() * h_q.element_size() + h_bt.numel() * 4 + h_cl.numel() * 4 +
                sum(k.numel() * k.element_size() * 2 + s.numel() * 8 for k, _, s in h_w) +
                (h_bm_t.numel() * 8 if h_bm_t is not None else 0))
         d2h = h_out.numel() * h_out.element_size()
@@ -358,7 +383,10 @@ def run_ours(args):
                 pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], d_bm, stream=stream)
             for dk, dv, ds in d_w:
                 write(dk, dv, ds)
-            decode(d_q, d_bt, d_cl)
+            if h_so is not None:  # the host schedule of this step, then its copy
+                h_so.numpy()[:] = pa.pa_prefix_order(h_bt.numpy(), h_cl.numpy())
+                d_so.copy_(h_so, non_blocking=True)
+            decode(d_q, d_bt, d_cl, d_so)
             h_out.copy_(out, non_blocking=True)
 
         for _ in range(min(args.warmup, 10)):
@@ -385,7 +413,8 @@ def run_ours(args):
     # Algorithmic bytes: KV of the referenced tokens; blocks shared by several
     # sequences (copy-on-write prefixes) count once, as the pool holds them once.
     kv_logical = W.kv_bytes(st, d, elem_bytes=sc.kv_elem_bytes, q_len=sc.q_len, window=sc.window)
-    kv = W.kv_bytes(st, d, unique=True, elem_bytes=sc.kv_elem_bytes) if args.workload == "cow" else kv_logical
+    kv = (W.kv_bytes(st, d, unique=True, elem_bytes=sc.kv_elem_bytes) if args.workload in ("cow", "prefix8b")
+          else kv_logical)
     algo = kv + W.qo_bytes(d, sc.q_len)
     peak, peak_kind = measured_hbm_peak()
     achieved = algo / (dec_avg_ms / 1e3) / 1e9
@@ -408,6 +437,9 @@ def run_ours(args):
                               f"max {int(st.context_lens.max())}",
                    "partition_tokens": P, "num_partitions": nparts,
                    **({"q_len": sc.q_len, "window": sc.window} if sc.ext else {}),
+                   **({"seq_order": "pa_prefix_order", "decode_ms_batch_order": no_order_ms,
+                       "decode_ms_prefix_order": dec_avg_ms,
+                       "prefix_order_speedup": no_order_ms / dec_avg_ms} if no_order_ms else {}),
                    "parallelism": f"{world} independent batches (one per GPU, no data-path collective)",
                    "l2": f"inputs larger than L2: {kv / 1e9:.2f} GB of KV read per step vs 126 MB L2",
                    "kv_bytes_per_step": kv, "kv_bytes_logical_per_step": kv_logical,

@@ -10,6 +10,8 @@
  *   pa_decode_fp8, pa_reshape_and_cache_fp8   the same over FP8 E4M3 caches
  *   pa_decode_ext         several query tokens per sequence and/or a sliding
  *                         window, over a 16-bit or FP8 cache
+ *   pa_prefix_cache_*, pa_prefix_order   host prefix cache (block-hash
+ *                         lookup) and the shared-prefix-aware decode order
  *   pa_decode             single-query attention of every sequence over its
  *                         cached tokens, gathered through its block table
  *
@@ -211,6 +213,11 @@ typedef struct pa_decode_opts {
     int32_t window; /* >= 0 tokens; 0 = no window */
     float k_scale;  /* K element = stored value * k_scale; finite, > 0 (1 for a plain cache) */
     float v_scale;  /* V element = stored value * v_scale; finite, > 0 */
+    const int32_t *seq_order; /* NULL, or a DEVICE permutation of [0, num_seqs): the order in which
+                                 sequences are scheduled (see pa_prefix_order); results do not
+                                 depend on it.  Entries outside [0, num_seqs) are skipped and
+                                 flagged (PA_DEVERR_CONTEXT); a sequence it does not list gets
+                                 no defined output */
 } pa_decode_opts;
 
 /* Workspace bytes pa_decode_ext needs (0 = none), (size_t)-1 for invalid
@@ -241,6 +248,57 @@ pa_status pa_decode_ext(void *out, const void *q, const void *k_cache, const voi
                         int32_t num_kv_heads, const pa_dims *dims, const pa_decode_opts *opts,
                         int32_t max_context_len, int32_t partition_tokens, void *workspace,
                         size_t workspace_bytes, void *stream);
+
+/*
+ * Prefix caching, host side ("vLLM PagedAttention 大模型推理架构深度实战"
+ * section 7.3: requests with an identical prefix are recognised and share
+ * KV-cache blocks; section 2.3: a block's reference count is the number of
+ * sequences mapping it).  A table from the content of a full 16-token block
+ * (its token ids, chained to the block holding the previous 16 tokens) to the
+ * physical block holding its K/V.  Host memory and host pointers only; not
+ * thread-safe (one owner, like the block manager that calls it).
+ *
+ * create:  a cache for block ids [0, num_blocks); NULL on error.
+ * match:   the longest chain of cached full blocks equal to the first tokens
+ *          of `tokens`; writes their ids to blocks_out (at most max_blocks),
+ *          takes one reference on each and returns how many (>= 0), or a
+ *          negative pa_status.
+ * insert:  registers the full blocks of a sequence (block i holds tokens
+ *          [16 i, 16 i + 16)); a block whose prefix is cached already is
+ *          left out (the cached one stays canonical); new entries hold one
+ *          reference (the inserting sequence's).
+ * release: drops one reference on each cached block given (others are
+ *          ignored); returns how many were cached.  A block with no
+ *          reference stays cached and becomes evictable.
+ * evict:   removes up to max_blocks evictable blocks, least recently
+ *          released first, writes their ids (free for reuse) and returns how
+ *          many.  Their descendants can no longer be matched.
+ * stats:   number of cached and evictable blocks, hits and lookups so far.
+ */
+typedef struct pa_prefix_cache pa_prefix_cache;
+pa_prefix_cache *pa_prefix_cache_create(int64_t num_blocks);
+void pa_prefix_cache_destroy(pa_prefix_cache *cache);
+int32_t pa_prefix_cache_match(pa_prefix_cache *cache, const int32_t *tokens, int32_t num_tokens,
+                              int32_t *blocks_out, int32_t max_blocks);
+pa_status pa_prefix_cache_insert(pa_prefix_cache *cache, const int32_t *tokens, int32_t num_tokens,
+                                 const int32_t *blocks, int32_t num_blocks);
+int32_t pa_prefix_cache_release(pa_prefix_cache *cache, const int32_t *blocks, int32_t num_blocks);
+int32_t pa_prefix_cache_evict(pa_prefix_cache *cache, int32_t max_blocks, int32_t *blocks_out);
+pa_status pa_prefix_cache_stats(const pa_prefix_cache *cache, int64_t *cached, int64_t *evictable,
+                                int64_t *hits, int64_t *lookups);
+
+/*
+ * Shared-prefix-aware schedule (host): order[i] = the i-th sequence decode
+ * should visit, grouping sequences that share their first block (and so
+ * their cached prefix) so that their CTAs run together and the shared
+ * blocks are read from HBM once and then served from L2.  Sort key: (first
+ * block id, sequence index); empty contexts last.  block_tables [num_seqs,
+ * max_blocks_per_seq] and context_lens are HOST arrays; order is a host
+ * array of num_seqs.  Pass it (copied to the device) as
+ * pa_decode_opts.seq_order.
+ */
+pa_status pa_prefix_order(const int32_t *block_tables, const int32_t *context_lens, int32_t num_seqs,
+                          int32_t max_blocks_per_seq, int32_t *order);
 
 /*
  * Cache write (ybb.press section 六, "write into the KV cache block").

@@ -29,6 +29,8 @@ FP8_CACHE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 # The C entry points declared in include/pa.h, in declaration order.
 EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", "pa_decode_noalloc",
            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_decode_ext_workspace_size", "pa_decode_ext",
+           "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_cache_match", "pa_prefix_cache_insert",
+           "pa_prefix_cache_release", "pa_prefix_cache_evict", "pa_prefix_cache_stats", "pa_prefix_order",
            "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_last_error", "pa_device_error",
            "pa_version"]
 
@@ -51,7 +53,7 @@ class pa_dims(ctypes.Structure):
 
 class pa_decode_opts(ctypes.Structure):
     _fields_ = [("q_len", ctypes.c_int32), ("window", ctypes.c_int32), ("k_scale", ctypes.c_float),
-                ("v_scale", ctypes.c_float)]
+                ("v_scale", ctypes.c_float), ("seq_order", ctypes.c_void_p)]
 
 
 def _load(path: str = LIB_PATH):
@@ -78,6 +80,24 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_ext_workspace_size.restype = u64
     lib.pa_decode_ext.argtypes = [vp, vp, vp, vp, vp, vp, f32, i32, dp, op, i32, i32, vp, u64, vp]
     lib.pa_decode_ext.restype = ctypes.c_int
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lp = ctypes.POINTER(ctypes.c_int64)
+    lib.pa_prefix_cache_create.argtypes = [i64]
+    lib.pa_prefix_cache_create.restype = vp
+    lib.pa_prefix_cache_destroy.argtypes = [vp]
+    lib.pa_prefix_cache_destroy.restype = None
+    lib.pa_prefix_cache_match.argtypes = [vp, ip, i32, ip, i32]
+    lib.pa_prefix_cache_match.restype = i32
+    lib.pa_prefix_cache_insert.argtypes = [vp, ip, i32, ip, i32]
+    lib.pa_prefix_cache_insert.restype = ctypes.c_int
+    lib.pa_prefix_cache_release.argtypes = [vp, ip, i32]
+    lib.pa_prefix_cache_release.restype = i32
+    lib.pa_prefix_cache_evict.argtypes = [vp, i32, ip]
+    lib.pa_prefix_cache_evict.restype = i32
+    lib.pa_prefix_cache_stats.argtypes = [vp, lp, lp, lp, lp]
+    lib.pa_prefix_cache_stats.restype = ctypes.c_int
+    lib.pa_prefix_order.argtypes = [ip, ip, i32, i32, ip]
+    lib.pa_prefix_order.restype = ctypes.c_int
     lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, dp, vp]
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [vp, vp, i32, vp, i32, dp, vp]
@@ -258,7 +278,8 @@ def ext_dims(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor)
 def pa_decode_ext(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                   block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, num_kv_heads: int,
                   max_context_len: int, q_len: int = 1, window: int = 0, k_scale: float = 1.0, v_scale: float = 1.0,
-                  partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                  partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+                  seq_order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Multi-token / sliding-window decode: q and out are [S, q_len, H, D];
     query i of sequence s sits at position context_lens[s] - q_len + i and
     attends to its `window` most recent positions (all when 0).  The caches
@@ -269,13 +290,91 @@ def pa_decode_ext(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_c
     if q.dim() != 4 or q.shape[1] != q_len or tuple(out.shape) != tuple(q.shape):
         raise ValueError("q and out must be [num_seqs, q_len, num_heads, head_dim]")
     dims = ext_dims(q, k_cache, block_tables)
-    opts = pa_decode_opts(int(q_len), int(window), float(k_scale), float(v_scale))
+    if seq_order is not None:
+        _need_cuda(seq_order)
+        if seq_order.dtype != torch.int32 or seq_order.numel() != q.shape[0]:
+            raise TypeError("seq_order must be int32 [num_seqs]")
+    opts = pa_decode_opts(int(q_len), int(window), float(k_scale), float(v_scale),
+                          None if seq_order is None else seq_order.data_ptr())
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = LIB.pa_decode_ext(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
                            float(scale), int(num_kv_heads), ctypes.byref(dims), ctypes.byref(opts),
                            int(max_context_len), int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
     _check(st)
     return out
+
+
+# ---------------------------------------------------------------------------
+# prefix caching (host)
+# ---------------------------------------------------------------------------
+def _i32p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+class PrefixCache:
+    """The library's host prefix cache (pa_prefix_cache_*): token ids of
+    full 16-token blocks -> the physical blocks holding their K/V."""
+
+    def __init__(self, num_blocks: int):
+        self._h = LIB.pa_prefix_cache_create(int(num_blocks))
+        if not self._h:
+            raise PagedAttentionError(-3, pa_last_error())
+
+    def close(self) -> None:
+        if self._h:
+            LIB.pa_prefix_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def match(self, tokens) -> list:
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        out = np.zeros(max(1, t.size // 16), dtype=np.int32)
+        n = LIB.pa_prefix_cache_match(self._h, _i32p(t), int(t.size), _i32p(out), int(t.size // 16))
+        if n < 0:
+            raise PagedAttentionError(n, pa_last_error())
+        return out[:n].tolist()
+
+    def insert(self, tokens, blocks) -> None:
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        b = np.ascontiguousarray(blocks, dtype=np.int32)
+        _check(LIB.pa_prefix_cache_insert(self._h, _i32p(t), int(t.size), _i32p(b), int(b.size)))
+
+    def release(self, blocks) -> int:
+        import numpy as np
+        b = np.ascontiguousarray(blocks, dtype=np.int32)
+        n = LIB.pa_prefix_cache_release(self._h, _i32p(b), int(b.size))
+        if n < 0:
+            raise PagedAttentionError(n, pa_last_error())
+        return int(n)
+
+    def evict(self, max_blocks: int) -> list:
+        import numpy as np
+        out = np.zeros(max(1, max_blocks), dtype=np.int32)
+        n = LIB.pa_prefix_cache_evict(self._h, int(max_blocks), _i32p(out))
+        if n < 0:
+            raise PagedAttentionError(n, pa_last_error())
+        return out[:n].tolist()
+
+    def stats(self) -> dict:
+        v = [ctypes.c_int64(0) for _ in range(4)]
+        _check(LIB.pa_prefix_cache_stats(self._h, *[ctypes.byref(x) for x in v]))
+        return dict(zip(("cached", "evictable", "hits", "lookups"), (x.value for x in v)))
+
+
+def pa_prefix_order(block_tables, context_lens):
+    """Host: the shared-prefix-aware order of the batch (numpy int32 [S])."""
+    import numpy as np
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = cl.shape[0]
+    MB = bt.shape[1] if bt.ndim == 2 else 0
+    order = np.zeros(max(1, S), dtype=np.int32)
+    _check(LIB.pa_prefix_order(_i32p(bt), _i32p(cl), int(S), int(MB), _i32p(order)))
+    return order[:S]
 
 
 def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -120,7 +120,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       const int32_t *block_tables, const int32_t *context_lens, float scale, float k_scale,
                       float v_scale, int32_t num_kv_heads, const pa_dims *dims, int32_t max_context_len,
                       int32_t partition_tokens, void *workspace, size_t workspace_bytes, void *stream,
-                      int32_t q_len = 1, int32_t window = 0) {
+                      int32_t q_len = 1, int32_t window = 0, const int32_t *seq_order = nullptr) {
     pa_status st;
     if (num_kv_heads != dims->num_kv_heads)
         return fail(PA_ERR_SHAPE, "num_kv_heads %d != dims->num_kv_heads %d", num_kv_heads, dims->num_kv_heads);
@@ -160,6 +160,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.group = g;
     p.q_len = q_len;
     p.window = window;
+    p.seq_order = seq_order;
     const int rows = row_capacity(g * q_len);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_fp8(dims);
@@ -254,7 +255,7 @@ pa_status pa_decode_ext(void *out, const void *q, const void *k_cache, const voi
     if (st != PA_OK) return st;
     return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, opts->k_scale, opts->v_scale,
                        num_kv_heads, dims, max_context_len, partition_tokens, workspace, workspace_bytes, stream,
-                       opts->q_len, opts->window);
+                       opts->q_len, opts->window, opts->seq_order);
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,

@@ -71,10 +71,14 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     int32_t *tbl = reinterpret_cast<int32_t *>(smem + S.table_off);
     __shared__ int fail_s;
 
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.x, kvh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads;
     const int head0 = kvh * G;  // unmasked launches only (group == G, q_len == 1)
+    pdl_launch_dependents();
+    pdl_wait();
+    const int s = scheduled_seq(p, blockIdx.z, part == 0 && kvh == 0 && tid == 0);
+    if (s < 0) return;
     // flat q / out row of row r: plain decode keeps the group's rows contiguous
     auto row_of = [&](int r) -> int64_t {
         if constexpr (kMasked) return query_row(p, s, kvh, r);
@@ -82,8 +86,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     };
     const int rows = kMasked ? p.group * p.q_len : G;  // real rows (the rest is padding)
 
-    pdl_launch_dependents();
-    pdl_wait();
     const SeqSplit sp = seq_split(p, s, part == 0 && kvh == 0 && tid == 0);
     const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part >= nparts) return;

@@ -30,6 +30,7 @@ struct DecodeParams {
     int32_t group;               // query heads per KV head
     int32_t q_len;               // query tokens per sequence (q, out: [S, q_len, H, D])
     int32_t window;              // sliding window in tokens, 0 = none
+    const int32_t *seq_order;    // nullptr, or the sequence each blockIdx.z visits
 };
 
 // Whether a launch needs per-row position masks (several query tokens or a

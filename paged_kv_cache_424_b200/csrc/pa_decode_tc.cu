@@ -30,6 +30,7 @@
 // = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
 // Results go to `out` (one partition) or to the split workspace for the
 // log-sum-exp merge, exactly like the CUDA-core kernel.
+#include <climits>
 #include <mutex>
 #include <type_traits>
 
@@ -143,18 +144,21 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
     int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
 
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.x, kvh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, head0 = kvh * G;  // head0: unmasked launches (group == G, q_len == 1)
     T *out = reinterpret_cast<T *>(p.out);
+    pdl_launch_dependents();
+    pdl_wait();
+    const int s = scheduled_seq(p, blockIdx.z, part == 0 && kvh == 0 && tid == 0);
+    if (s < 0) return;
+    // flat q / out row of row r: plain decode keeps the group's rows contiguous
     auto row_of = [&](int r) -> int64_t {
         if constexpr (kMasked) return query_row(p, s, kvh, r);
         return (int64_t)s * H + head0 + r;
     };
     const int rows = kMasked ? p.group * p.q_len : G;
 
-    pdl_launch_dependents();
-    pdl_wait();
     const SeqSplit sp = seq_split(p, s, part == 0 && kvh == 0 && tid == 0);
     const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part >= nparts) return;
@@ -258,16 +262,12 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
         }
         const int t = tid;                                      // token of S, dim of O
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // TMEM lane quadrant
-        int lo[G], hi[G];  // attended positions of each column (masked launches)
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            if constexpr (kMasked) {
-                row_range(p, L, h, &lo[h], &hi[h]);
-            } else {
-                lo[h] = 0;
-                hi[h] = L - 1;
-            }
-        }
+        // masked launches: column h is query token h >> lg, whose position is
+        // hi0 + (h >> lg); it attends (position - window, position] (all
+        // positions up to its own without a window); padding columns none
+        const int hi0 = L - p.q_len;
+        const int lg = 31 - __clz(p.group);
+        const int win = p.window > 0 ? p.window : INT_MAX;
         float m[G], l[G], acc[G], alpha_prev[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -298,7 +298,10 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     bool live = valid;
-                    if constexpr (kMasked) live = live && tok >= lo[h] && tok <= hi[h];
+                    if constexpr (kMasked) {
+                        const int pos = hi0 + (h >> lg);
+                        live = live && h < rows && tok <= pos && pos - tok < win;
+                    }
                     x[h] = live ? sv[h] * p.scale_log2 : -INFINITY;
                     exceed |= x[h] > m[h] + kLazyMax;
                 }

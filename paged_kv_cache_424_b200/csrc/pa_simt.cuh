@@ -46,6 +46,18 @@ __device__ __forceinline__ int64_t checked_block(const DecodeParams &p, int32_t 
     return b;
 }
 
+// The sequence CTA row z works on: z itself, or seq_order[z]; -1 (flagged)
+// for an entry outside the batch.
+__device__ __forceinline__ int scheduled_seq(const DecodeParams &p, int z, bool report) {
+    if (!p.seq_order) return z;
+    const int s = p.seq_order[z];
+    if (s < 0 || s >= p.num_seqs) {
+        if (report) flag_error(PA_DEVERR_CONTEXT);
+        return -1;
+    }
+    return s;
+}
+
 // First table entry any query of a sequence of L tokens reads: 0, or with a
 // sliding window the block holding the earliest attended position (that of
 // query token 0, L - q_len - window + 1).

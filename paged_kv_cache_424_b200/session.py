@@ -82,11 +82,16 @@ class DeviceSession:
 
     def decode_inputs(self, step: Step) -> Dict[str, torch.Tensor]:
         d = self.sc.dims
-        return {
+        inp = {
             "q": to_device(step.q, d.dtype, self.device),
             "block_tables": torch.from_numpy(step.block_tables).to(self.device),
             "context_lens": torch.from_numpy(step.context_lens).to(self.device),
         }
+        if self.sc.prefix_order:
+            # the host schedule: sequences sharing a prefix next to each other
+            order = pa.pa_prefix_order(step.block_tables, step.context_lens)
+            inp["seq_order"] = torch.from_numpy(order).to(self.device)
+        return inp
 
     def write_inputs(self, step: Step):
         d = self.sc.dims
@@ -156,7 +161,7 @@ class DeviceSession:
         out4 = out if out.dim() == 4 else out[:, None]
         pa.pa_decode_ext(out4, q4, self.k_cache, self.v_cache, inp["block_tables"], inp["context_lens"], sc.scale,
                          sc.dims.num_kv_heads, maxlen, sc.q_len, sc.window, sc.k_scale, sc.v_scale, P, ws,
-                         stream=stream)
+                         stream=stream, seq_order=inp.get("seq_order"))
         return out
 
     def run_step(self, step: Step, partition_tokens: Optional[int] = None) -> torch.Tensor:

@@ -147,10 +147,12 @@ class Scenario:
     # positions.
     q_len: int = 1
     window: int = 0
+    # decode in the shared-prefix-aware order (pa_prefix_order / seq_order)
+    prefix_order: bool = False
 
     @property
     def ext(self) -> bool:
-        return self.q_len != 1 or self.window != 0
+        return self.q_len != 1 or self.window != 0 or self.prefix_order
 
     @property
     def kv_elem_bytes(self) -> int:
@@ -354,8 +356,11 @@ def long70b(seed: int = 3, num_seqs: int = 8, context_len: int = 32768, num_bloc
 
 def cow(seed: int = 4, num_prompts: int = 16, samples: int = 8, prefix: int = 1000,
         max_tail: int = 256, num_blocks: int = 8192, cow_every_sample: bool = False,
-        v_lo: float = -1.0) -> Scenario:
-    """Parallel sampling: prefixes shared by ``samples`` sequences each."""
+        v_lo: float = -1.0, shuffle: bool = False, name: str = "cow") -> Scenario:
+    """Parallel sampling: prefixes shared by ``samples`` sequences each.
+    With ``shuffle`` the batch lists the sequences in a seeded random order
+    (as a scheduler admitting requests over time would), so sharers of one
+    prefix are scattered through the batch."""
     rng = np.random.default_rng(seed)
     S = num_prompts * samples
     mb = -(-(prefix + max_tail + 1) // BLOCK_SIZE)
@@ -373,6 +378,8 @@ def cow(seed: int = 4, num_prompts: int = 16, samples: int = 8, prefix: int = 10
         kids = [b.bm.fork(parent) for _ in range(samples)]
         b.bm.free_sequence(parent)
         seqs.extend(kids)
+    if shuffle:
+        seqs = [seqs[i] for i in rng.permutation(S)]
     tails = rng.integers(0, max_tail + 1, size=S)
     tail_slots, dec_slots = [], []
     for s, t in zip(seqs, tails):
@@ -389,11 +396,21 @@ def cow(seed: int = 4, num_prompts: int = 16, samples: int = 8, prefix: int = 10
     writes = [Write(k1, v1, np.asarray(tail_slots, np.int64)),
               Write(k2, v2, np.asarray(dec_slots, np.int64))]
     st = b.step(seqs, writes)
-    return Scenario("cow", dims, _scale(128), b.pad_block, [st],
+    return Scenario(name, dims, _scale(128), b.pad_block, [st],
                     note=f"{num_prompts} prompts x {samples} samples, prefix {prefix}, tails "
                          f"U[0,{max_tail}], H=32/Hk=8, D=128, bf16, pool {num_blocks}, "
-                         f"{'copy per sample' if cow_every_sample else 'copy while shared'}",
+                         f"{'copy per sample' if cow_every_sample else 'copy while shared'}"
+                         f"{', shuffled batch order' if shuffle else ''}",
                     shared_blocks=np.asarray(shared, np.int64))
+
+
+def prefix8b(seed: int = 7, num_prompts: int = 64, samples: int = 8, prefix: int = 2000, max_tail: int = 64,
+             num_blocks: int = 16384, shuffle: bool = True, v_lo: float = -1.0) -> Scenario:
+    """Shared prefixes larger than L2: 64 prompts of 2000 tokens (500 MiB of
+    K/V on the 8B shape), each shared by 8 sequences listed in a shuffled
+    batch order; decode visits them in the order pa_prefix_order gives."""
+    sc = cow(seed, num_prompts, samples, prefix, max_tail, num_blocks, v_lo=v_lo, shuffle=shuffle, name="prefix8b")
+    return replace(sc, prefix_order=True, note=sc.note + ", decoded in shared-prefix order")
 
 
 def spec8b(seed: int = 5, num_seqs: int = 256, q_len: int = 4, median: int = 1024, cap: int = 4096,
@@ -440,7 +457,7 @@ def with_fp8_cache(sc: Scenario, k_scale: float = FP8_K_SCALE, v_scale: float = 
 
 
 SCENARIOS = {"tiny": tiny, "mha7b": mha7b, "gqa8b": gqa8b, "long70b": long70b, "cow": cow, "spec8b": spec8b,
-             "window70b": window70b}
+             "window70b": window70b, "prefix8b": prefix8b}
 CONFIG_ORDER = ["tiny", "mha7b", "gqa8b", "long70b", "cow"]
 
 

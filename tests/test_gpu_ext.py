@@ -181,3 +181,43 @@ def test_window70b_fp8_multi_token_reduced():
     sc = W().with_fp8_cache(W().window70b(seed=64, num_seqs=2, context_len=3000, window=257, q_len=2,
                                           num_blocks=1024))
     run_and_compare(sc)
+
+
+# ---------------------------------------------------------------------------
+# shared-prefix order (pa_prefix_order -> pa_decode_opts.seq_order)
+# ---------------------------------------------------------------------------
+def test_prefix8b_reduced_order_is_bit_identical_to_batch_order():
+    import dataclasses
+    from paged_kv_cache_424_b200.session import DeviceSession
+    sc = W().prefix8b(seed=71, num_prompts=4, num_blocks=2048)
+    run_and_compare(sc)                                   # in prefix order, against the oracle
+    st = sc.steps[0]
+    a = DeviceSession(sc).run_step(st)
+    b = DeviceSession(dataclasses.replace(sc, prefix_order=False)).run_step(st)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)), "the schedule changed the results"
+
+
+def test_prefix8b_full_sampled():
+    sc = W().prefix8b()
+    seqs = np.sort(np.random.default_rng(72).choice(sc.dims.num_seqs, 10, replace=False))
+    run_and_compare(sc, seqs=seqs)
+
+
+@pytest.mark.parametrize("g", [1, 4])
+def test_seq_order_entry_outside_the_batch_is_skipped_and_flagged(g):
+    from paged_kv_cache_424_b200 import binding as pa
+    rng = np.random.default_rng(73 + g)
+    p = Paged(rng, [40, 70, 300, 5], 2 * g, 2, 128, "f16")
+    q = _dev16(p.q, "f16")[:, None]
+    k, v = _dev16(p.k_cache, "f16"), _dev16(p.v_cache, "f16")
+    bt, cl = torch.from_numpy(p.tables).cuda(), torch.from_numpy(p.lens).cuda()
+    ref = torch.empty_like(q)
+    pa.pa_decode_ext(ref, q, k, v, bt, cl, 0.1, 2, 300)
+    order = torch.tensor([2, 0, 9, 1], dtype=torch.int32, device="cuda")   # 9 is not a sequence; 3 is missing
+    out = torch.zeros_like(q)
+    pa.pa_decode_ext(out, q, k, v, bt, cl, 0.1, 2, 300, seq_order=order)
+    assert pa.pa_device_error() & 2, "out-of-range entry not flagged"
+    for s in (0, 1, 2):
+        assert torch.equal(out[s].view(torch.int16), ref[s].view(torch.int16))
+    assert torch.all(out[3] == 0), "the skipped CTA row wrote something"
