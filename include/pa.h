@@ -182,8 +182,12 @@ pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const
  * weights ("vLLM PagedAttention 大模型推理架构深度实战" section 5.2) and
  * KV-cache compression as a goal (section 九 item 3).  Same definition as
  * pa_decode with K_s[j] = decode(k code) * k_scale and V_s[j] = decode(v code)
- * * v_scale; q / out in dims->dtype.  Runs on the CUDA-core kernel for every
- * group size; workspace as from pa_decode_workspace_size with the same dims.
+ * * v_scale; q / out in dims->dtype.  Groups of 4, 8 or 16 query heads at
+ * head_dim 128 run on the tensor-core kernel (codes widened in shared
+ * memory to f16, q converted to f16 for the MMA: a bf16 q must lie within
+ * f16's range, |q| <= 65504, and loses precision below 2^-14); other shapes
+ * on the CUDA-core kernel.
+ * Workspace as from pa_decode_workspace_size with the same dims.
  */
 pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
                         const int32_t *block_tables, const int32_t *context_lens, float scale,

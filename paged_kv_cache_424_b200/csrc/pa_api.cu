@@ -80,6 +80,16 @@ int row_capacity(int rows) {
     return c;
 }
 
+// Row capacity of the tensor-core kernel for these dims, or 0 for the
+// CUDA-core kernel: GQA groups (and multi-token queries) of 4 rows or more
+// at head_dim 128, where the CUDA-core kernel turns ALU-bound, for 16-bit
+// and FP8 caches alike.  With 1 or 2 rows the CUDA-core kernel is faster
+// (measured on B200: over an FP8 cache 122 us against 273 us for the 7B MHA
+// batch, whose rows would pad the MMA's 16 columns).
+int tc_rows(const pa_dims *d, int rows) {
+    return pa::decode_tc_supported(d->head_dim, rows, d->num_blocks, d->num_kv_heads) ? rows : 0;
+}
+
 pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
                     int32_t q_len = 1, int32_t window = 0) {
     if (max_context_len < 0) return fail(PA_ERR_SHAPE, "max_context_len %d < 0", max_context_len);
@@ -90,8 +100,7 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
                     partition_tokens, kMaxPartitionTokens);
     const int g = d->num_heads / d->num_kv_heads;
-    const int rows = row_capacity(g * q_len);
-    const bool tc = !kv_fp8(d) && pa::decode_tc_supported(d->head_dim, rows, d->num_blocks, d->num_kv_heads);
+    const bool tc = tc_rows(d, row_capacity(g * q_len)) != 0;
     const int P = partition_tokens != 0 ? partition_tokens : tc ? kAutoPartitionTc : kAutoPartitionSimt;
     int ctx_blocks = (max_context_len + 15) / 16;
     if (window > 0) {
@@ -162,11 +171,11 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.window = window;
     p.seq_order = seq_order;
     const int rows = row_capacity(g * q_len);
+    const int tc = tc_rows(dims, rows);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_fp8(dims);
-    cudaError_t e = !fp8 && pa::decode_tc_supported(dims->head_dim, rows, dims->num_blocks, dims->num_kv_heads)
-                        ? pa::launch_decode_tc(p, dims->dtype, rows, cs)
-                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, rows, fp8, cs);
+    cudaError_t e = tc ? pa::launch_decode_tc(p, dims->dtype, tc, fp8, cs)
+                       : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, rows, fp8, cs);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "pa_decode_fp8 launch" : "pa_decode launch");
     return PA_OK;
 }

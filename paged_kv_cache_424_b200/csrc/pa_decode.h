@@ -69,7 +69,7 @@ cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_d
 // Tensor-core decode for row capacities 4, 8 or 16 at head_dim 128 (GQA
 // groups, or several query tokens) and whether it applies to these sizes.
 bool decode_tc_supported(int head_dim, int rows, int64_t num_blocks, int num_kv_heads);
-cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, bool fp8_cache, cudaStream_t stream);
 
 // Cache kernels.
 struct CacheDims {

@@ -9,19 +9,21 @@
 //   O^T (128 dims x 16)  = V^T (128 x 128 tokens) . P^T (128 x 16)  [PV]
 // (the G query rows padded to the MMA's N = 16).
 //
-// CTA = (partition, KV head, sequence): 7 warps.
-//   warp 4  K producer and warp 6  V producer: per chunk, 2-D tiled TMA loads
+// CTA = (partition, KV head, sequence): 7 warps (11 with 16 columns, whose
+// softmax work is split over 8 warps, 8 columns each).
+//   warp 4  K producer and warp 6  V producer (8 and 10 with 16 columns): per chunk, 2-D tiled TMA loads
 //           of the 8 blocks' K (or V) rows (16 rows x 64 dims per box,
 //           128-byte swizzle) into the K (or V) tile, as soon as the previous
 //           chunk's MMA that read the tile has completed; blocks past the
 //           partition are loaded from an out-of-range row, which the TMA
 //           fills with zeros.  The partition's table slice is read once, 32
 //           entries per coalesced load.
-//   warp 5  MMA issuer (one thread): S into TMEM (double-buffered), then
+//   warp 5  MMA issuer (warp 9 with 16 columns; one thread): S into TMEM (double-buffered), then
 //           O = V^T P^T into TMEM (double-buffered), each completion signalled
 //           by tcgen05.commit on an mbarrier; allocates / frees TMEM.
 //   warps 0-3 softmax: thread t owns TMEM lane t = token t of S and output
-//           dim t of O.  Masks tokens past the context, keeps the online
+//           dim t of O (with 16 columns warps 0-7: warps w and w + 4 share
+//           lane quadrant w and take columns 0-7 and 8-15).  Masks tokens past the context, keeps the online
 //           softmax with a lazy running max (raised only when some logit
 //           beats it by 2^8; a CTA-wide flag skips the max reduction in all
 //           other chunks), writes P (same 16-bit type as V) into a swizzled
@@ -47,7 +49,6 @@ constexpr int kD = 128;
 constexpr int kN = 16;              // MMA N: query heads padded to 16
 constexpr int kChunk = 128;         // tokens per chunk (MMA M)
 constexpr int kChunkBlocks = kChunk / kBlock;
-constexpr int kThreadsTc = 224;
 constexpr int kRegion = kChunk * 128;   // one 64-dim half of a K or V tile (bytes)
 
 // Shared-memory layout (bytes from the 1024-aligned base).
@@ -57,7 +58,7 @@ constexpr int kQOff = kVOff + 2 * kRegion;      // 65536
 constexpr int kPOff = kQOff + 2 * kN * 128;     // 69632
 constexpr int kRedOff = kPOff + 2 * kN * 128;   // 73728: [2][4][16] floats
 constexpr int kBarOff = kRedOff + 2 * 4 * kN * 4;
-constexpr int kNumBars = 10;
+constexpr int kNumBars = 12;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;  // TMEM base, fail flag, 4 lazy-max flags
 constexpr int kSmemTc = kMiscOff + 32;
 
@@ -76,7 +77,11 @@ __device__ __forceinline__ bool wait_ok(uint64_t *bar, uint32_t parity, int *fai
     return false;
 }
 
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier 1 over the N softmax threads.
+template <int N>
+__device__ __forceinline__ void softmax_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -118,19 +123,102 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
     }
 }
 
-// CTAs per SM: 3 (registers and shared memory both allow it) except for
-// groups of 16, whose per-thread state needs the registers of 2.
+// Softmax warps: one per TMEM lane quadrant, each thread holding the state
+// of every column; with 16 columns two warps per quadrant, each owning 8 of
+// the columns, so a thread's state stays that of 8 columns.  Then the K
+// producer, the MMA issuer and the V producer.
+__host__ __device__ constexpr int tc_soft_warps(int G) { return G > 8 ? 8 : 4; }
+__host__ __device__ constexpr int tc_threads(int G) { return (tc_soft_warps(G) + 3) * 32; }
+// FP8 E4M3 caches: the producer loads a chunk's codes (128 tokens x 128
+// bytes) by TMA into the second 64-dim region of the 16-bit tile and
+// converts them there into the tile's f16 layout (codes widen exactly to
+// f16).  A step reads 4 rows of codes (512 contiguous bytes, one 16-byte
+// load per lane) before it writes those 4 rows of f16: a row's f16 lands in
+// both regions at the same row, over its own codes only, so no code is
+// overwritten before it is read.
+__device__ __forceinline__ void convert_fp8_chunk(unsigned char *tile, int lane) {
+    const unsigned char *codes = tile + kRegion;
+    const int c16 = lane & 7;  // codes [16 c16, 16 c16 + 16) of the row = dims
+    unsigned char *dst = tile + (c16 >> 2) * kRegion;
+    const int col = (c16 & 3) * 16;  // first element of those dims within their region
+#pragma unroll 4
+    for (int step = 0; step < kChunk / 4; ++step) {
+        const int r = step * 4 + (lane >> 3);
+        const uint4 raw = *reinterpret_cast<const uint4 *>(codes + r * 128 + c16 * 16);
+        __syncwarp();  // all 4 rows read before any of them is overwritten
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] & 0xffffu), __NV_E4M3);
+            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] >> 16), __NV_E4M3);
+            h[2 * j] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+            h[2 * j + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+        }
+        *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
+        __syncwarp();
+    }
+}
+
+// The producer of an FP8 tile: per chunk, wait until the MMA that read the
+// tile's previous chunk has completed, load the chunk's codes into the
+// tile's second region (`stage` completes the copies), convert, and arrive
+// on `full` (32 arrivals: one per lane).
+__device__ __forceinline__ void produce_tile_fp8(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
+                                                 uint64_t *stage, uint64_t *full, uint64_t *empty, int *fail, int s,
+                                                 int kvh, int b0, int nb, int nch, int oob_row, int lane) {
+    const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
+    auto window = [&](int w) -> int {
+        const int bi = w * 32 + lane;
+        return bi < nb ? (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock) : oob_row;
+    };
+    if (lane == 0) prefetch_tmap(tmap);
+    int cur = window(0);
+    int next = nb > 32 ? window(1) : oob_row;
+    for (int c = 0; c < nch; ++c) {
+        if (c > 0 && (c & 3) == 0) {
+            cur = next;
+            next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1) : oob_row;
+        }
+        const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
+        bool ok = true;
+        if (lane == 0) {
+            ok = c == 0 || wait_ok(empty, (c - 1) & 1, fail);
+            if (ok) mbar_arrive_expect_tx(stage, kChunk * 128);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane < kChunkBlocks) tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 0, y, stage);
+        if (!__all_sync(0xffffffffu, wait_ok(stage, c & 1, fail))) break;
+        convert_fp8_chunk(tile, lane);
+        fence_proxy_async_smem();  // the f16 tile is read by the MMA (async proxy)
+        mbar_arrive(full);
+    }
+}
+
+// CTAs per SM: 3 (registers and shared memory both allow it) except with 16
+// columns, whose 11 warps fit twice.
 __host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; }
 
 // G: columns of S (query rows per KV head: the group, or group x query
 // tokens with kMasked, padded to a power of two).
-template <typename T, int G, bool kMasked>
-__global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
+// kFp8: the caches hold E4M3 codes; K, V, Q and P tiles are f16 and the
+// MMA runs f16 x f16 (q converted to f16 on load), k_scale sits in
+// scale_log2 and v_scale multiplies the output.
+template <typename T, int G, bool kMasked, bool kFp8>
+__global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
+    static_assert(!kFp8 || kMasked, "FP8 launches take the masked variant (it applies v_scale)");
     using E = Elem<T>;
-    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    constexpr int kCols = G <= 8 ? 8 : 16;  // live TMEM columns of S and O
+    using MT = typename std::conditional<kFp8, __half, T>::type;  // type of the MMA operands
+    using EM = Elem<MT>;
+    constexpr bool kBf16 = std::is_same<MT, __nv_bfloat16>::value;
+    constexpr int kSW = tc_soft_warps(G);       // softmax warps
+    constexpr int kST = kSW * 32;                // softmax threads
+    constexpr int kGT = G > 8 ? 8 : G;           // columns per softmax thread
+    constexpr int kWarpK = kSW, kWarpMma = kSW + 1, kWarpV = kSW + 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *k_t = smem + kKOff;
     unsigned char *v_t = smem + kVOff;
@@ -140,6 +228,7 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
     uint64_t *k_full = bars + 0, *k_empty = bars + 1, *v_full = bars + 2, *v_empty = bars + 3;
     uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8, *q_full = bars + 9;
+    uint64_t *k_stage = bars + 10, *v_stage = bars + 11;  // FP8: codes landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMiscOff);
     int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
     int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
@@ -179,23 +268,25 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
 
     // ---- set-up -----------------------------------------------------------------
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tc::tmem_alloc(tmem_slot, kTmemCols);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
         *fail = 0;
         for (int i = 0; i < 4; ++i) lazy_flag[i] = 0;
-        mbar_init(k_full, 1);
+        mbar_init(k_full, kFp8 ? 32 : 1);  // FP8: the producer's 32 lanes after converting
         mbar_init(k_empty, 1);
-        mbar_init(v_full, 1);
+        mbar_init(v_full, kFp8 ? 32 : 1);
         mbar_init(v_empty, 1);
+        mbar_init(k_stage, 1);
+        mbar_init(v_stage, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         mbar_init(&o_full[0], 1);
         mbar_init(&o_full[1], 1);
-        mbar_init(p_full, 128);
-        mbar_init(q_full, 128);
+        mbar_init(p_full, kST);
+        mbar_init(q_full, kST);
         fence_mbar_init();
     }
     tc::fence_before_sync();
@@ -203,11 +294,17 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
-        produce_tile(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-    } else if (warp == 6) {
-        produce_tile(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-    } else if (warp == 5) {
+    if (warp == kWarpK) {
+        if constexpr (kFp8)
+            produce_tile_fp8(p, &tmap_k, k_t, k_stage, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        else
+            produce_tile(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+    } else if (warp == kWarpV) {
+        if constexpr (kFp8)
+            produce_tile_fp8(p, &tmap_v, v_t, v_stage, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        else
+            produce_tile(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+    } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc_qk = tc::instr_desc_f16(kBf16, false, kChunk, kN);
@@ -251,105 +348,120 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
             // K-major 128-byte swizzle, two 64-dim regions.  Loaded while the
             // producers already stream K and V.
             const T *q = reinterpret_cast<const T *>(p.q);
-            for (int i = tid; i < kN * (kD / 8); i += 128) {
+            for (int i = tid; i < kN * (kD / 8); i += kST) {
                 const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (r < rows) v = *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + c16 * 8);
+                if constexpr (kFp8 && !std::is_same<T, __half>::value) {
+                    // bf16 q -> f16 for the f16 MMA (exact for 2^-14 <= |q| <= 65504)
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = E::to_float2(w[j]);
+                        const __half2 hh = __floats2half2_rn(f.x, f.y);
+                        w[j] = *reinterpret_cast<const uint32_t *>(&hh);
+                    }
+                    v = make_uint4(w[0], w[1], w[2], w[3]);
+                }
                 *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
             }
             fence_proxy_async_smem();
             mbar_arrive(q_full);
         }
-        const int t = tid;                                      // token of S, dim of O
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // TMEM lane quadrant
+        const int t = tid & 127;                                      // token of S, dim of O
+        const int c0 = kSW == 8 ? (warp >> 2) * kGT : 0;              // this thread's first column
+        const uint32_t lane_base = (uint32_t)((kSW == 8 ? warp & 3 : warp) * 32) << 16;  // TMEM lane quadrant
         // masked launches: column h is query token h >> lg, whose position is
         // hi0 + (h >> lg); it attends (position - window, position] (all
         // positions up to its own without a window); padding columns none
         const int hi0 = L - p.q_len;
         const int lg = 31 - __clz(p.group);
         const int win = p.window > 0 ? p.window : INT_MAX;
-        float m[G], l[G], acc[G], alpha_prev[G];
+        // per-thread state of columns c0 + j, j < kGT
+        float m[kGT], l[kGT], acc[kGT], alpha_prev[kGT];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            m[h] = -INFINITY;
-            l[h] = 0.f;
-            acc[h] = 0.f;
-            alpha_prev[h] = 1.f;
+        for (int j = 0; j < kGT; ++j) {
+            m[j] = -INFINITY;
+            l[j] = 0.f;
+            acc[j] = 0.f;
+            alpha_prev[j] = 1.f;
         }
         auto epilogue = [&](int c) {
             if (!wait_ok(&o_full[c & 1], (c >> 1) & 1, fail)) return;
             tc::fence_after_sync();
-            float o[kCols];
-            tc::tmem_ld<kCols>(tmem + lane_base + o_col(c & 1), o);
+            float o[8];
+            tc::tmem_ld<8>(tmem + lane_base + o_col(c & 1) + c0, o);
 #pragma unroll
-            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha_prev[h], o[h]);
+            for (int j = 0; j < kGT; ++j) acc[j] = fmaf(acc[j], alpha_prev[j], o[j]);
         };
         const bool has_tail = (b0 + nb == nblk) && (L % kBlock) != 0;  // partial last block here
         for (int c = 0; c < nch; ++c) {
-            float x[G];
+            float x[kGT];
             const int tok = tok0 + c * kChunk + t;
             const bool valid = tok < tok_end;
             bool ok = wait_ok(&s_full[c & 1], (c >> 1) & 1, fail);
             bool exceed = false;
             if (ok) {
                 tc::fence_after_sync();
-                float sv[kCols];
-                tc::tmem_ld<kCols>(tmem + lane_base + s_col(c & 1), sv);
+                float sv[8];
+                tc::tmem_ld<8>(tmem + lane_base + s_col(c & 1) + c0, sv);
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
+                for (int j = 0; j < kGT; ++j) {
                     bool live = valid;
                     if constexpr (kMasked) {
+                        const int h = c0 + j;
                         const int pos = hi0 + (h >> lg);
                         live = live && h < rows && tok <= pos && pos - tok < win;
                     }
-                    x[h] = live ? sv[h] * p.scale_log2 : -INFINITY;
-                    exceed |= x[h] > m[h] + kLazyMax;
+                    x[j] = live ? sv[j] * p.scale_log2 : -INFINITY;
+                    exceed |= x[j] > m[j] + kLazyMax;
                 }
             } else {
 #pragma unroll
-                for (int h = 0; h < G; ++h) x[h] = -INFINITY;
+                for (int j = 0; j < kGT; ++j) x[j] = -INFINITY;
             }
             // Lazy running max: a CTA-wide flag says whether any logit of the
             // chunk beats its head's running max by more than 2^8; only then
             // are the per-head chunk maxima reduced and the state rescaled.
             if (__any_sync(0xffffffffu, exceed) && lane == 0) lazy_flag[c & 3] = 1;
-            softmax_sync();
+            softmax_sync<kST>();
             const bool update = lazy_flag[c & 3] != 0;
-            if (t == 0) lazy_flag[(c + 2) & 3] = 0;  // slot of chunk c + 2: its readers are done
-            float alpha[G];
+            if (tid == 0) lazy_flag[(c + 2) & 3] = 0;  // slot of chunk c + 2: its readers are done
+            float alpha[kGT];
 #pragma unroll
-            for (int h = 0; h < G; ++h) alpha[h] = 1.f;
-            if (update) {  // uniform across the 128 threads
-                float *rc = red + (c & 1) * 4 * kN;
+            for (int j = 0; j < kGT; ++j) alpha[j] = 1.f;
+            if (update) {  // uniform across the softmax threads
+                float *rc = red + (c & 1) * 4 * kN;  // [quadrant][column]
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float v = x[h];
+                for (int j = 0; j < kGT; ++j) {
+                    float v = x[j];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                    if (lane == 0) rc[warp * kN + h] = v;
+                    if (lane == 0) rc[(kSW == 8 ? warp & 3 : warp) * kN + c0 + j] = v;
                 }
-                softmax_sync();
+                softmax_sync<kST>();
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
+                for (int j = 0; j < kGT; ++j) {
+                    const int h = c0 + j;
                     const float cm = fmaxf(fmaxf(rc[h], rc[kN + h]), fmaxf(rc[2 * kN + h], rc[3 * kN + h]));
-                    if (cm > m[h] + kLazyMax) {
-                        alpha[h] = ex2(m[h] - cm);  // 0 on the first chunk (m = -inf)
-                        l[h] *= alpha[h];
-                        m[h] = cm;
+                    if (cm > m[j] + kLazyMax) {
+                        alpha[j] = ex2(m[j] - cm);  // 0 on the first chunk (m = -inf)
+                        l[j] *= alpha[j];
+                        m[j] = cm;
                     }
                 }
             }
-            T pv[G];
+            MT pv[kGT];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+            for (int j = 0; j < kGT; ++j) {
                 // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
-                pv[h] = (kMasked && x[h] == -INFINITY) ? E::from_float(0.f) : E::from_float(ex2(x[h] - m[h]));
-                l[h] += E::to_float(pv[h]);  // the rounded weight the MMA sees
+                pv[j] = (kMasked && x[j] == -INFINITY) ? EM::from_float(0.f) : EM::from_float(ex2(x[j] - m[j]));
+                l[j] += EM::to_float(pv[j]);  // the rounded weight the MMA sees
             }
             if (c > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
 #pragma unroll
-            for (int h = 0; h < G; ++h) alpha_prev[h] = alpha[h];
-            if (c == nch - 1 && has_tail && ok) {
+            for (int j = 0; j < kGT; ++j) alpha_prev[j] = alpha[j];
+            if (c == nch - 1 && has_tail && ok && c0 == 0) {
                 // Rows of the partial last block past the context come from the
                 // pool and may hold anything (NaN): zero them in the V tile
                 // once it has landed, so 0 * V stays 0 in the PV product.
@@ -361,12 +473,15 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
                             *reinterpret_cast<uint4 *>(v_t + j * kRegion + t * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            // P tile: K-major, rows = heads, columns = tokens (two 64-token regions)
+            // P tile: K-major, rows = heads, columns = tokens (two 64-token
+            // regions); this thread writes rows c0 .. c0 + (16 / (kSW / 4)) - 1
+            // (its columns, then zero rows up to 16)
             unsigned char *pr = p_t + (t >> 6) * (kN * 128);
+            constexpr int kRowsW = kN / (kSW / 4);
 #pragma unroll
-            for (int h = 0; h < kN; ++h) {
-                const T v = h < G ? pv[h < G ? h : 0] : E::from_float(0.f);
-                *reinterpret_cast<T *>(pr + tc::sw128_offset(h, t & 63)) = v;
+            for (int j = 0; j < kRowsW; ++j) {
+                const MT v = j < kGT ? pv[j < kGT ? j : 0] : EM::from_float(0.f);
+                *reinterpret_cast<MT *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
@@ -376,39 +491,40 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
 
         // l: per-thread partial sums over this thread's tokens -> total per head
         float *rl = red;  // both halves of the chunk-max buffer are free now
-        softmax_sync();
+        softmax_sync<kST>();
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float v = l[h];
+        for (int j = 0; j < kGT; ++j) {
+            float v = l[j];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) rl[warp * kN + h] = v;
+            if (lane == 0) rl[(kSW == 8 ? warp & 3 : warp) * kN + c0 + j] = v;
         }
-        softmax_sync();
+        softmax_sync<kST>();
         if (!is_failed(fail)) {
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+            for (int j = 0; j < kGT; ++j) {
+                const int h = c0 + j;
                 const float lt = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
                 if constexpr (kMasked) {
                     if (h >= rows) break;
                     // lt = 0 only for a column with no position in this partition
-                    const float o = lt > 0.f ? acc[h] / lt * p.v_scale : 0.f;
+                    const float o = lt > 0.f ? acc[j] / lt * p.v_scale : 0.f;
                     const int64_t qr = row_of(h);
                     if (direct) {
                         out[qr * kD + t] = E::from_float(o);
                     } else {
                         const int64_t r = qr * p.max_parts + part;
                         p.ws_o[r * kD + t] = o;
-                        if (t == 0) p.ws_lse[r] = lt > 0.f ? m[h] + log2f(lt) : -INFINITY;
+                        if (t == 0) p.ws_lse[r] = lt > 0.f ? m[j] + log2f(lt) : -INFINITY;
                     }
                 } else {  // plain decode: every column has tokens, V unscaled
-                    const float o = acc[h] / lt;
+                    const float o = acc[j] / lt;
                     if (direct) {
                         out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
                     } else {
                         const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
                         p.ws_o[r * kD + t] = o;
-                        if (t == 0) p.ws_lse[r] = m[h] + log2f(lt);
+                        if (t == 0) p.ws_lse[r] = m[j] + log2f(lt);
                     }
                 }
             }
@@ -418,7 +534,7 @@ __global__ void __launch_bounds__(kThreadsTc, tc_ctas_per_sm(G))
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 5) tc::tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMma) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -443,6 +559,20 @@ EncodeTiledFn encode_fn() {
 
 // A cache [NB, Hk, 16, 128] seen as rows of 128 elements; boxes of 16 rows
 // x 64 elements with the 128-byte swizzle; out-of-range rows read as zero.
+// An FP8 cache [NB, Hk, 16, 128] seen as rows of 128 one-byte codes; boxes
+// of 16 rows x 128 bytes, unswizzled (the producer converts them).
+bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD};
+    const cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_cache_map(CUtensorMap *map, const void *base, int64_t rows, bool bf16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -456,14 +586,15 @@ bool encode_cache_map(CUtensorMap *map, const void *base, int64_t rows, bool bf1
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int G, bool kMasked>
+template <typename T, int G, bool kMasked, bool kFp8 = false>
 cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
     CUtensorMap tk, tv;
-    if (!encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) ||
-        !encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value))
-        return cudaErrorInvalidValue;
-    auto kern = decode_tc_kernel<T, G, kMasked>;
+    const bool ok = kFp8 ? encode_code_map(&tk, p.k_cache, rows) && encode_code_map(&tv, p.v_cache, rows)
+                         : encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) &&
+                               encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value);
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = decode_tc_kernel<T, G, kMasked, kFp8>;
     static int configured[kMaxDevices] = {};
     static int carveout_set[kMaxDevices] = {};
     int dev = 0;
@@ -476,7 +607,7 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     }
     e = ensure_smem(kern, kSmemTc, configured);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(kThreadsTc), kSmemTc, stream, p, tk, tv,
+    e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(tc_threads(G)), kSmemTc, stream, p, tk, tv,
                    (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
@@ -495,7 +626,18 @@ cudaError_t launch_tc_m(const DecodeParams &p, int rows, cudaStream_t stream) {
 // The plain variant neither masks nor scales V: anything else takes the
 // masked one (with q_len = 1, no window its masks keep every token).
 template <typename T>
-cudaError_t launch_tc_d(const DecodeParams &p, int rows, cudaStream_t stream) {
+cudaError_t launch_tc_fp8(const DecodeParams &p, int rows, cudaStream_t stream) {
+    switch (rows) {
+        case 4: return launch_tc_t<T, 4, true, true>(p, stream);
+        case 8: return launch_tc_t<T, 8, true, true>(p, stream);
+        case 16: return launch_tc_t<T, 16, true, true>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t launch_tc_d(const DecodeParams &p, int rows, bool fp8, cudaStream_t stream) {
+    if (fp8) return launch_tc_fp8<T>(p, rows, stream);
     return decode_masked(p) || p.v_scale != 1.f ? launch_tc_m<T, true>(p, rows, stream)
                                                 : launch_tc_m<T, false>(p, rows, stream);
 }
@@ -507,8 +649,9 @@ bool decode_tc_supported(int head_dim, int rows, int64_t num_blocks, int num_kv_
            num_blocks * num_kv_heads * kBlock < ((int64_t)1 << 31) - kBlock;
 }
 
-cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, cudaStream_t stream) {
-    return dtype == PA_F16 ? launch_tc_d<__half>(p, rows, stream) : launch_tc_d<__nv_bfloat16>(p, rows, stream);
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, int rows, bool fp8_cache, cudaStream_t stream) {
+    return dtype == PA_F16 ? launch_tc_d<__half>(p, rows, fp8_cache, stream)
+                           : launch_tc_d<__nv_bfloat16>(p, rows, fp8_cache, stream);
 }
 
 }  // namespace pa

@@ -85,12 +85,14 @@ def test_bad_dims_rejected(lib, kw, status):
     assert lib.pa_last_error()
 
 
-def test_fp8_cache_plans_on_the_cuda_core_kernel(lib):
-    # group 4 / head_dim 128 would take the tensor-core kernel (1024-token
-    # partitions) over a 16-bit cache; an FP8 cache takes the CUDA-core one (512)
-    d = _dims(lib, kv_dtype=lib.PA_FP8_E4M3)
-    assert lib.pa_decode_num_partitions(d, 1024, 0) == 2
-    assert lib.pa_decode_num_partitions(d, 4096, 0) == 8
+def test_fp8_cache_plan_follows_the_kernel(lib):
+    # groups of 4+ at head_dim 128 take the tensor-core kernel (1024-token
+    # partitions) over FP8 caches too; MHA and head_dim 64 the CUDA-core one (512)
+    f8 = lib.PA_FP8_E4M3
+    assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=f8), 1024, 0) == 1
+    assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=f8), 4096, 0) == 4
+    assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=f8, num_heads=8), 1024, 0) == 2
+    assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=f8, head_dim=64), 1024, 0) == 2
     assert lib.pa_decode_num_partitions(_dims(lib, kv_dtype=lib.PA_BF16), 1024, 0) == 1
 
 
