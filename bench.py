@@ -9,8 +9,15 @@ context spans several 512-token partitions).  Default workload: the
 Llama-2-7B-shaped MHA batch (64 sequences, lengths U[128, 2048], 32 heads,
 head_dim 128, fp16, 16384-block pool).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--kv 16|fp8]
   python bench.py --impl reference ...      # the CPU oracle, timed the same way
+
+Other workloads: gqa8b, long70b, cow (the pages' other shapes), spec8b (4
+query tokens per sequence, pa_decode_ext), window70b (4096-token sliding
+window), prefix8b (shared prefixes in a shuffled batch, decoded in the
+pa_prefix_order schedule; the batch-order time is reported beside), swap
+(pa_swap_blocks device <-> pinned host).  --kv fp8 runs a workload over an
+FP8 E4M3 cache (pa_reshape_and_cache_fp8 + pa_decode_fp8).
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch of
 the same shape (sequences are independent; no collective on the data path),
