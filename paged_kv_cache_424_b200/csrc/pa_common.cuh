@@ -52,9 +52,22 @@ struct E4M3 {
     uint8_t code;
 };
 
+// Two E4M3 codes (element 0 in the low byte) -> f16x2 bits (element 0 in
+// the low half), exactly: one cvt (PTX ISA, cvt with .e4m3x2 source, sm_89+).
+__device__ __forceinline__ uint32_t e4m3x2_to_half2_bits(uint16_t pair) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(pair));
+    return r;
+}
+
+// The two 16-bit halves of a 32-bit word (a register split, no arithmetic).
+__device__ __forceinline__ void split_b32(uint32_t w, uint16_t &lo, uint16_t &hi) {
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+}
+
 // Two E4M3 codes (element 0 in the low byte) -> two floats, exactly.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t pair) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    const uint32_t h = e4m3x2_to_half2_bits(pair);
     return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 

@@ -150,10 +150,10 @@ __device__ __forceinline__ void convert_fp8_chunk(unsigned char *tile, int lane)
         uint32_t h[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] & 0xffffu), __NV_E4M3);
-            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] >> 16), __NV_E4M3);
-            h[2 * j] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-            h[2 * j + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+            uint16_t lo, hi;
+            split_b32(w[j], lo, hi);
+            h[2 * j] = e4m3x2_to_half2_bits(lo);
+            h[2 * j + 1] = e4m3x2_to_half2_bits(hi);
         }
         *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col)) = make_uint4(h[0], h[1], h[2], h[3]);
         *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col + 8)) = make_uint4(h[4], h[5], h[6], h[7]);

@@ -248,8 +248,10 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
             float k[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const float2 lo = e4m3x2_to_float2((uint16_t)(w[j] & 0xffffu));
-                const float2 hi = e4m3x2_to_float2((uint16_t)(w[j] >> 16));
+                uint16_t l16, h16;
+                split_b32(w[j], l16, h16);
+                const float2 lo = e4m3x2_to_float2(l16);
+                const float2 hi = e4m3x2_to_float2(h16);
                 k[4 * j] = lo.x; k[4 * j + 1] = lo.y; k[4 * j + 2] = hi.x; k[4 * j + 3] = hi.y;
             }
             fma8(k, 2 * c);
@@ -293,8 +295,10 @@ __device__ __forceinline__ void simt_block(SimtState<D, G> &st, const unsigned c
         if constexpr (kFp8) {
             if constexpr (kPV == 4) {
                 const uint32_t raw = *reinterpret_cast<const uint32_t *>(vs + tok * D + lane * 4);
-                const float2 a = e4m3x2_to_float2((uint16_t)(raw & 0xffffu));
-                const float2 b = e4m3x2_to_float2((uint16_t)(raw >> 16));
+                uint16_t l16, h16;
+                split_b32(raw, l16, h16);
+                const float2 a = e4m3x2_to_float2(l16);
+                const float2 b = e4m3x2_to_float2(h16);
                 vf[0] = a.x;
                 vf[1] = a.y;
                 vf[2] = b.x;
