@@ -353,6 +353,17 @@ pa_status pa_swap_blocks(const void *src_k, const void *src_v, int64_t src_num_b
                          void *dst_v, int64_t dst_num_blocks, const int64_t *block_mapping,
                          int32_t num_pairs, const pa_dims *dims, void *stream);
 
+/*
+ * Diagnostic of the failure path: enqueues on `stream` one kernel whose
+ * single pipeline wait can never complete (an mbarrier nothing arrives on),
+ * bounded to about `milliseconds` (1..2000) of SM clock at the device's
+ * maximum clock rate.  The wait gives up, sets PA_DEVERR_TIMEOUT in the
+ * device error word and the kernel returns: the context stays usable.  Every
+ * pipeline wait of the decode kernels is bounded the same way (about 2 s).
+ * Read the word with pa_device_error.
+ */
+pa_status pa_check_wait_timeout(int32_t milliseconds, void *stream);
+
 /* Thread-local description of the last non-OK status returned on this
  * thread ("" if none).  Owned by the library; valid until the next call. */
 const char *pa_last_error(void);

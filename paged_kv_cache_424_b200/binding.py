@@ -31,8 +31,8 @@ EXPORTS = ["pa_decode_workspace_size", "pa_decode_num_partitions", "pa_decode", 
            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_decode_ext_workspace_size", "pa_decode_ext",
            "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_cache_match", "pa_prefix_cache_insert",
            "pa_prefix_cache_release", "pa_prefix_cache_evict", "pa_prefix_cache_stats", "pa_prefix_order",
-           "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_last_error", "pa_device_error",
-           "pa_version"]
+           "pa_reshape_and_cache", "pa_copy_blocks", "pa_swap_blocks", "pa_check_wait_timeout", "pa_last_error",
+           "pa_device_error", "pa_version"]
 
 
 class LibraryMissing(RuntimeError):
@@ -106,6 +106,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_last_error.argtypes = []
     lib.pa_last_error.restype = ctypes.c_char_p
+    lib.pa_check_wait_timeout.argtypes = [i32, vp]
+    lib.pa_check_wait_timeout.restype = ctypes.c_int
     lib.pa_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.pa_device_error.restype = ctypes.c_int
     lib.pa_version.argtypes = []
@@ -438,6 +440,12 @@ def pa_swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor
                             int(dst_k.shape[0]), _ptr(block_mapping), int(block_mapping.numel() // 2),
                             ctypes.byref(dims), _stream(stream))
     _check(st)
+
+
+def pa_check_wait_timeout(milliseconds: int = 50, stream=None) -> None:
+    """Enqueue the bounded-wait diagnostic (a wait that can never complete
+    gives up after about `milliseconds` and flags PA_DEVERR_TIMEOUT)."""
+    _check(LIB.pa_check_wait_timeout(int(milliseconds), _stream(stream)))
 
 
 def pa_device_error(stream=None) -> int:

@@ -363,6 +363,18 @@ pa_status pa_swap_blocks(const void *src_k, const void *src_v, int64_t src_num_b
     return PA_OK;
 }
 
+pa_status pa_check_wait_timeout(int32_t milliseconds, void *stream) {
+    if (milliseconds < 1 || milliseconds > 2000)
+        return fail(PA_ERR_SHAPE, "milliseconds %d must be in [1, 2000]", milliseconds);
+    int dev = 0, khz = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+    if (e != cudaSuccess || khz <= 0) return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidValue, "clock rate");
+    e = pa::launch_wait_timeout_probe((long long)khz * milliseconds, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_check_wait_timeout launch");
+    return PA_OK;
+}
+
 pa_status pa_device_error(void *stream, uint32_t *word) {
     if (!word) return fail(PA_ERR_NULL, "word is NULL");
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -159,7 +159,24 @@ __global__ void __launch_bounds__(256)
     quantize16(value + src, v_scale, v_cache + dst);
 }
 
+// Diagnostic: one thread waits on an mbarrier that nothing ever arrives on,
+// with a bound of `limit_cycles` SM cycles; the bounded wait gives up, sets
+// PA_DEVERR_TIMEOUT and the kernel returns.  The same wait (with its longer
+// default bound) guards every pipeline stage of the decode kernels.
+__global__ void wait_timeout_probe_kernel(long long limit_cycles) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, limit_cycles);  // never completes: no arrival
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t stream) {
+    wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
                                          const int64_t *slot_mapping, int32_t num_tokens, const CacheDims &d,

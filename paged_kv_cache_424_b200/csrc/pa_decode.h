@@ -86,6 +86,7 @@ cudaError_t launch_reshape_and_cache_fp8(const void *key, const void *value, voi
 cudaError_t launch_copy_blocks(void *const *k_caches, void *const *v_caches, int32_t num_layers,
                                const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
                                cudaStream_t stream);
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t stream);
 cudaError_t launch_swap_blocks(const void *src_k, const void *src_v, int64_t src_blocks, void *dst_k, void *dst_v,
                                int64_t dst_blocks, const int64_t *block_mapping, int32_t num_pairs, const CacheDims &d,
                                cudaStream_t stream);

@@ -166,6 +166,8 @@ assert L.pa_copy_blocks(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctyp
 assert L.pa_copy_blocks(None, None, 0, None, 0, ctypes.byref(d), None) == 0
 assert L.pa_copy_blocks(None, None, 1, p, -1, ctypes.byref(d), None) == -3
 assert L.pa_device_error(None, None) == -1
+assert L.pa_check_wait_timeout(0, None) == -3
+assert L.pa_check_wait_timeout(3000, None) == -3
 
 # FP8 E4M3 caches: entry point and kv_dtype must agree; scales must be positive
 f8 = dims(kv_dtype=lib.PA_FP8_E4M3)
