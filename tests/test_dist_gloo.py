@@ -38,7 +38,15 @@ def _worker(rank: int, world: int, port: int, q):
         # each rank builds its own batch: same shape, different contents
         sc = bench.make_scenario("mha7b", seed=1 + rank, num_seqs=4, num_blocks=2048)
         st = sc.steps[0]
-        q.put((rank, t_max, st.q.shape, st.block_tables.shape, int(st.q[0, 0, 0]), st.context_lens.tolist()))
+        # the extension workloads shard the same way: per-rank batches of one shape
+        ext = []
+        for name, kw in (("spec8b", dict(num_seqs=4, num_blocks=2048)), ("prefix8b", dict(num_seqs=16, num_blocks=1024)),
+                         ("window70b", dict(num_seqs=1, num_blocks=4096))):
+            e = bench.make_scenario(name, seed=1 + rank, **kw).steps[0]
+            ext.append((name, e.q.shape, e.block_tables.shape, int(e.q.reshape(-1)[0])))
+        fp8 = bench.make_scenario("gqa8b", seed=1 + rank, num_seqs=4, num_blocks=4096, kv="fp8")
+        q.put((rank, t_max, st.q.shape, st.block_tables.shape, int(st.q[0, 0, 0]), st.context_lens.tolist(), ext,
+               fp8.kv_dtype))
     finally:
         dist.destroy_process_group()
 
@@ -58,6 +66,10 @@ def test_two_ranks_max_time_and_independent_batches():
     assert [o[1] for o in out] == [11.0, 11.0], "max over ranks"
     assert out[0][2] == out[1][2] and out[0][3] == out[1][3], "same batch shape on every rank"
     assert out[0][5] != out[1][5] or out[0][4] != out[1][4], "ranks must decode different batches"
+    for (n0, qs0, bs0, v0), (n1, qs1, bs1, v1) in zip(out[0][6], out[1][6]):
+        assert n0 == n1 and qs0 == qs1 and bs0 == bs1, f"{n0}: ranks differ in shape"
+        assert v0 != v1, f"{n0}: ranks must decode different batches"
+    assert out[0][7] == out[1][7] == "fp8"
 
 
 def test_rank_count_mismatch_is_refused(monkeypatch):
