@@ -203,30 +203,37 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
 
 // out[row, :] = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p,
 // over the partitions sequence s actually uses (all -inf: a masked row with
-// no position, zero).  One CTA of D threads per (query token x head, s).
+// no position, zero).  A CTA of D threads takes `rows_per_cta` consecutive
+// rows (query token x head) of sequence s, so a batch with many rows pays
+// the per-sequence check and the launch once per group of rows.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p, const int rows_per_cta) {
     const int s = blockIdx.y, d = threadIdx.x;
     pdl_launch_dependents();
     pdl_wait();
     const SeqSplit sp = seq_split(p, s, false);
     const int nparts = sp.nparts;
     if (nparts <= 1) return;  // written directly by the decode kernel
-    const int64_t qr = (int64_t)s * p.q_len * p.num_heads + blockIdx.x;
-    const int64_t row = qr * p.max_parts;
-    const float *lse = p.ws_lse + row;
-    float M = -INFINITY;
-    for (int i = 0; i < nparts; ++i) M = fmaxf(M, lse[i]);
-    float wsum = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < nparts; ++i) {
-            const float w = exp2f(lse[i] - M);
-            wsum += w;
-            o = fmaf(w, p.ws_o[(row + i) * D + d], o);
+    const int rows = p.q_len * p.num_heads;
+    const int r0 = blockIdx.x * rows_per_cta;
+    const int r1 = min(r0 + rows_per_cta, rows);
+    for (int r = r0; r < r1; ++r) {
+        const int64_t qr = (int64_t)s * rows + r;
+        const int64_t row = qr * p.max_parts;
+        const float *lse = p.ws_lse + row;
+        float M = -INFINITY;
+        for (int i = 0; i < nparts; ++i) M = fmaxf(M, lse[i]);
+        float wsum = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+            for (int i = 0; i < nparts; ++i) {
+                const float w = exp2f(lse[i] - M);
+                wsum += w;
+                o = fmaf(w, p.ws_o[(row + i) * D + d], o);
+            }
+            o /= wsum;
         }
-        o /= wsum;
+        reinterpret_cast<T *>(p.out)[qr * D + d] = Elem<T>::from_float(o);
     }
-    reinterpret_cast<T *>(p.out)[qr * D + d] = Elem<T>::from_float(o);
 }
 
 template <typename T, typename KT, int D, int G, bool kMasked>
@@ -269,12 +276,18 @@ cudaError_t launch_part_k(const DecodeParams &p, int head_dim, int group, cudaSt
 }  // namespace
 
 cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream) {
-    const dim3 grid(p.num_heads * p.q_len, p.num_seqs);
+    // Rows per CTA: 1 while the grid stays under ~4 waves of small CTAs,
+    // up to 8 for batches with many rows (multi-token queries).
+    const int64_t rows = (int64_t)p.num_heads * p.q_len;
+    const int64_t total = rows * p.num_seqs;
+    int rpc = 1;
+    while (rpc < 8 && total / (rpc * 2) >= 8192) rpc *= 2;
+    const dim3 grid((unsigned)((rows + rpc - 1) / rpc), p.num_seqs);
     if (dtype == PA_F16)
-        return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, dim3(64), 0, stream, p)
-                              : launch_pdl(merge_part_kernel<__half, 128>, grid, dim3(128), 0, stream, p);
-    return head_dim == 64 ? launch_pdl(merge_part_kernel<__nv_bfloat16, 64>, grid, dim3(64), 0, stream, p)
-                          : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p);
+        return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, dim3(64), 0, stream, p, rpc)
+                              : launch_pdl(merge_part_kernel<__half, 128>, grid, dim3(128), 0, stream, p, rpc);
+    return head_dim == 64 ? launch_pdl(merge_part_kernel<__nv_bfloat16, 64>, grid, dim3(64), 0, stream, p, rpc)
+                          : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p, rpc);
 }
 
 cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int rows, bool fp8_cache,
