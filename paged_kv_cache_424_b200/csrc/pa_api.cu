@@ -90,6 +90,32 @@ int tc_rows(const pa_dims *d, int rows) {
     return pa::decode_tc_supported(d->head_dim, rows, d->num_blocks, d->num_kv_heads) ? rows : 0;
 }
 
+// Multiprocessors of the current device (148 on B200 if it does not answer).
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        return n;
+    cudaGetLastError();
+    return 148;
+}
+
+// Partitions one tensor-core CTA streams back to back: partitions shorter
+// than 1024 tokens (8 chunks) that start on a chunk are grouped up to 1024
+// tokens per CTA, which saves the per-CTA set-up (TMEM, barriers, Q tile,
+// pipeline fill; measured: the 70B shape at 512-token partitions ran at
+// 0.78 of the copy roofline against 0.87 at 1024), as long as the grid
+// keeps at least two waves of resident CTAs.  Each partition still gets its
+// own partial and the merge is unchanged.
+int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows) {
+    if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= 64) return 1;
+    const int64_t slots = (int64_t)sm_count() * (rows > 8 ? 2 : 3);
+    const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
+    int ppc = 64 / pl.part_blocks;
+    while (ppc > 1 && pairs * ((pl.max_parts + ppc - 1) / ppc) < 2 * slots) ppc >>= 1;
+    return ppc;
+}
+
 pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
                     int32_t q_len = 1, int32_t window = 0) {
     if (max_context_len < 0) return fail(PA_ERR_SHAPE, "max_context_len %d < 0", max_context_len);
@@ -172,6 +198,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.seq_order = seq_order;
     const int rows = row_capacity(g * q_len);
     const int tc = tc_rows(dims, rows);
+    p.parts_per_cta = tc ? tc_parts_per_cta(pl, dims->num_seqs, dims->num_kv_heads, tc) : 1;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_fp8(dims);
     cudaError_t e = tc ? pa::launch_decode_tc(p, dims->dtype, tc, fp8, cs)

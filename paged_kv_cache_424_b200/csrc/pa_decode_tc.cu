@@ -233,13 +233,17 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
     int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
 
-    const int part = blockIdx.x, kvh = blockIdx.y;
+    const int kvh = blockIdx.y;
+    // this CTA streams partitions part0 .. part0 + ppc - 1 (those that exist)
+    // back to back: one set-up, one pipeline, one partial per partition
+    const int ppc = p.parts_per_cta;
+    const int part0 = blockIdx.x * ppc;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, head0 = kvh * G;  // head0: unmasked launches (group == G, q_len == 1)
     T *out = reinterpret_cast<T *>(p.out);
     pdl_launch_dependents();
     pdl_wait();
-    const int s = scheduled_seq(p, blockIdx.z, part == 0 && kvh == 0 && tid == 0);
+    const int s = scheduled_seq(p, blockIdx.z, part0 == 0 && kvh == 0 && tid == 0);
     if (s < 0) return;
     // flat q / out row of row r: plain decode keeps the group's rows contiguous
     auto row_of = [&](int r) -> int64_t {
@@ -248,9 +252,10 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     };
     const int rows = kMasked ? p.group * p.q_len : G;
 
-    const SeqSplit sp = seq_split(p, s, part == 0 && kvh == 0 && tid == 0);
+    const SeqSplit sp = seq_split(p, s, part0 == 0 && kvh == 0 && tid == 0);
     const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
-    if (part >= nparts) return;
+    if (part0 >= nparts) return;
+    const int nmine = min(ppc, nparts - part0);  // partitions of this CTA
     const bool direct = nparts == 1;
     if (L == 0) {
         for (int i = tid; i < rows * kD; i += blockDim.x) out[row_of(i / kD) * kD + i % kD] = E::from_float(0.f);
@@ -261,9 +266,12 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
         if (tid == 0) flag_error(PA_DEVERR_LAYOUT);
         return;
     }
-    const int b0 = sp.bfirst + part * p.part_blocks;
-    const int nb = min(p.part_blocks, nblk - b0);          // blocks of this partition
+    const int b0 = sp.bfirst + part0 * p.part_blocks;
+    const int nb = min(nmine * p.part_blocks, nblk - b0);  // blocks of this CTA's partitions
     const int nch = (nb + kChunkBlocks - 1) / kChunkBlocks; // chunks of 128 tokens
+    // chunks per partition: partitions of several chunks start on a chunk
+    // (the host sets ppc > 1 only when part_blocks is a multiple of 8)
+    const int cpp = ppc > 1 ? p.part_blocks / kChunkBlocks : nch;
     const int tok0 = b0 * kBlock;
     const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
 
@@ -395,9 +403,68 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             for (int j = 0; j < kGT; ++j) acc[j] = fmaf(acc[j], alpha_prev[j], o[j]);
         };
         const bool has_tail = (b0 + nb == nblk) && (L % kBlock) != 0;  // partial last block here
+        // the partial of partition part0 + pi: per-column sums over the 4
+        // lane quadrants, then o = acc / l (and lse) to the output or the
+        // workspace; the last sync frees `red` for the next chunk's maxima
+        auto finalize = [&](int pi) {
+            float *rl = red;
+            softmax_sync<kST>();
+#pragma unroll
+            for (int j = 0; j < kGT; ++j) {
+                float v = l[j];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) rl[(kSW == 8 ? warp & 3 : warp) * kN + c0 + j] = v;
+            }
+            softmax_sync<kST>();
+            const int part = part0 + pi;
+            if (!is_failed(fail)) {
+#pragma unroll
+                for (int j = 0; j < kGT; ++j) {
+                    const int h = c0 + j;
+                    const float lt = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
+                    if constexpr (kMasked) {
+                        if (h >= rows) break;
+                        // lt = 0 only for a column with no position in this partition
+                        const float o = lt > 0.f ? acc[j] / lt * p.v_scale : 0.f;
+                        const int64_t qr = row_of(h);
+                        if (direct) {
+                            out[qr * kD + t] = E::from_float(o);
+                        } else {
+                            const int64_t r = qr * p.max_parts + part;
+                            p.ws_o[r * kD + t] = o;
+                            if (t == 0) p.ws_lse[r] = lt > 0.f ? m[j] + log2f(lt) : -INFINITY;
+                        }
+                    } else {  // plain decode: every column has tokens, V unscaled
+                        const float o = acc[j] / lt;
+                        if (direct) {
+                            out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
+                        } else {
+                            const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
+                            p.ws_o[r * kD + t] = o;
+                            if (t == 0) p.ws_lse[r] = m[j] + log2f(lt);
+                        }
+                    }
+                }
+            }
+            softmax_sync<kST>();
+        };
         for (int c = 0; c < nch; ++c) {
             float x[kGT];
             const int tok = tok0 + c * kChunk + t;
+            const int cl = c % cpp;  // chunk index within its partition
+            if (cl == 0 && c > 0) {
+                // chunk c - 1 closed a partition: finish and write it, start afresh
+                epilogue(c - 1);
+                finalize(c / cpp - 1);
+#pragma unroll
+                for (int j = 0; j < kGT; ++j) {
+                    m[j] = -INFINITY;
+                    l[j] = 0.f;
+                    acc[j] = 0.f;
+                    alpha_prev[j] = 1.f;
+                }
+            }
             const bool valid = tok < tok_end;
             bool ok = wait_ok(&s_full[c & 1], (c >> 1) & 1, fail);
             bool exceed = false;
@@ -458,7 +525,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 pv[j] = (kMasked && x[j] == -INFINITY) ? EM::from_float(0.f) : EM::from_float(ex2(x[j] - m[j]));
                 l[j] += EM::to_float(pv[j]);  // the rounded weight the MMA sees
             }
-            if (c > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
+            if (cl > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
 #pragma unroll
             for (int j = 0; j < kGT; ++j) alpha_prev[j] = alpha[j];
             if (c == nch - 1 && has_tail && ok && c0 == 0) {
@@ -488,47 +555,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             mbar_arrive(p_full);
         }
         epilogue(nch - 1);
-
-        // l: per-thread partial sums over this thread's tokens -> total per head
-        float *rl = red;  // both halves of the chunk-max buffer are free now
-        softmax_sync<kST>();
-#pragma unroll
-        for (int j = 0; j < kGT; ++j) {
-            float v = l[j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) rl[(kSW == 8 ? warp & 3 : warp) * kN + c0 + j] = v;
-        }
-        softmax_sync<kST>();
-        if (!is_failed(fail)) {
-#pragma unroll
-            for (int j = 0; j < kGT; ++j) {
-                const int h = c0 + j;
-                const float lt = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
-                if constexpr (kMasked) {
-                    if (h >= rows) break;
-                    // lt = 0 only for a column with no position in this partition
-                    const float o = lt > 0.f ? acc[j] / lt * p.v_scale : 0.f;
-                    const int64_t qr = row_of(h);
-                    if (direct) {
-                        out[qr * kD + t] = E::from_float(o);
-                    } else {
-                        const int64_t r = qr * p.max_parts + part;
-                        p.ws_o[r * kD + t] = o;
-                        if (t == 0) p.ws_lse[r] = lt > 0.f ? m[j] + log2f(lt) : -INFINITY;
-                    }
-                } else {  // plain decode: every column has tokens, V unscaled
-                    const float o = acc[j] / lt;
-                    if (direct) {
-                        out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
-                    } else {
-                        const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
-                        p.ws_o[r * kD + t] = o;
-                        if (t == 0) p.ws_lse[r] = m[j] + log2f(lt);
-                    }
-                }
-            }
-        }
+        finalize((nch - 1) / cpp);
     }
 
     tc::fence_before_sync();
@@ -607,7 +634,8 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     }
     e = ensure_smem(kern, kSmemTc, configured);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(tc_threads(G)), kSmemTc, stream, p, tk, tv,
+    e = launch_pdl(kern, dim3((p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, p.num_kv_heads, p.num_seqs),
+                   dim3(tc_threads(G)), kSmemTc, stream, p, tk, tv,
                    (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);

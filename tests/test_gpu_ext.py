@@ -221,3 +221,36 @@ def test_seq_order_entry_outside_the_batch_is_skipped_and_flagged(g):
     for s in (0, 1, 2):
         assert torch.equal(out[s].view(torch.int16), ref[s].view(torch.int16))
     assert torch.all(out[3] == 0), "the skipped CTA row wrote something"
+
+
+# ---------------------------------------------------------------------------
+# several partitions per tensor-core CTA (partitions of 128-512 tokens on a
+# grid of 512 (sequence, KV head) pairs, enough for the host to group them)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("P", [128, 256, 384, 512])
+def test_several_partitions_per_tensor_core_cta(orc, P):
+    from paged_kv_cache_424_b200 import binding as pa
+    rng = np.random.default_rng(500 + P)
+    S, Hk, g = 64, 8, 4
+    lens = rng.integers(1, 2001, size=S)
+    lens[:4] = [1, 127, 128, 129]
+    p = Paged(rng, lens, Hk * g, Hk, 128, "bf16")
+    scale = 0.088
+    ref = p.run(orc, scale)
+    q = _dev16(p.q, "bf16")
+    k, v = _dev16(p.k_cache, "bf16"), _dev16(p.v_cache, "bf16")
+    bt, cl = torch.from_numpy(p.tables).cuda(), torch.from_numpy(p.lens).cuda()
+    maxlen = int(lens.max())
+    dims = pa.dims_of(q, k, bt)
+    n = pa.pa_decode_workspace_size(dims, maxlen, P)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
+    out = torch.full_like(q, float("nan"))
+    pa.pa_decode(out, q, k, v, bt, cl, scale, Hk, maxlen, P, ws)
+    torch.cuda.synchronize()
+    compare(out, ref, "bf16", f"P={P}")
+    # masked: 2 query tokens and a window, same grouping
+    q2 = rand_bits(rng, (S, 2, Hk * g, 128), "bf16")
+    ref2 = orc.paged_decode_ext(q2, p.k_cache, p.v_cache, p.tables, p.lens, scale, "bf16", 2, 700)
+    tables = poison_before_window(p.tables, lens, 2, 700)
+    out2 = run_ext(q2, p.k_cache, p.v_cache, tables, lens, scale, "bf16", 2, 700, P)
+    compare(out2, ref2, "bf16", f"masked P={P}")
