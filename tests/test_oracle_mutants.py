@@ -91,19 +91,40 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutant_is_caught(name, tmp_path):
+def _run_mutant(name: str, workdir: str) -> tuple:
+    """Build mutant `name` and run the pins on it in a child process:
+    returns (returncode, stdout, stderr)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert old in src, f"mutant {name}: pattern no longer in the oracle source"
-    path = tmp_path / "mutant.c"
-    path.write_text(src.replace(old, new))
-    lib = oracle.build(str(path), str(tmp_path / "libmutant.so"))
+    if old not in src:
+        return (None, "", f"mutant {name}: pattern no longer in the oracle source")
+    path = os.path.join(workdir, f"{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib = oracle.build(path, os.path.join(workdir, f"lib{name}.so"))
     tests = os.path.dirname(os.path.abspath(__file__))
     code = _CHILD.format(tests=tests, root=os.path.dirname(tests), lib=lib)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600,
                        env={**os.environ, "OMP_NUM_THREADS": "2"})
-    if r.returncode < 0:
+    return (r.returncode, r.stdout, r.stderr)
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's child run, several at once (each in its own process)."""
+    import concurrent.futures as cf
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    jobs = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
+        futs = {name: ex.submit(_run_mutant, name, workdir) for name in MUTANTS}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, mutant_results):
+    rc, out, err = mutant_results[name]
+    assert rc is not None, err
+    if rc < 0:
         return  # killed by a signal (an out-of-bounds access): caught
-    assert r.returncode == 0, r.stderr[-2000:]
-    assert "PASSED_ALL" not in r.stdout, f"mutant {name} passed every pin"
+    assert rc == 0, err[-2000:]
+    assert "PASSED_ALL" not in out, f"mutant {name} passed every pin"
