@@ -132,31 +132,39 @@ __host__ __device__ constexpr int tc_threads(int G) { return (tc_soft_warps(G) +
 // FP8 E4M3 caches: the producer loads a chunk's codes (128 tokens x 128
 // bytes) by TMA into the second 64-dim region of the 16-bit tile and
 // converts them there into the tile's f16 layout (codes widen exactly to
-// f16).  A step reads 4 rows of codes (512 contiguous bytes, one 16-byte
-// load per lane) before it writes those 4 rows of f16: a row's f16 lands in
-// both regions at the same row, over its own codes only, so no code is
-// overwritten before it is read.
+// f16).  A step reads 16 rows of codes (four 512-byte runs, four
+// independent 16-byte loads per lane) before it writes those 16 rows of
+// f16: a row's f16 lands in both regions at the same row, over its own codes
+// only, so no code is overwritten before it is read.
 __device__ __forceinline__ void convert_fp8_chunk(unsigned char *tile, int lane) {
     const unsigned char *codes = tile + kRegion;
     const int c16 = lane & 7;  // codes [16 c16, 16 c16 + 16) of the row = dims
     unsigned char *dst = tile + (c16 >> 2) * kRegion;
     const int col = (c16 & 3) * 16;  // first element of those dims within their region
-#pragma unroll 4
-    for (int step = 0; step < kChunk / 4; ++step) {
-        const int r = step * 4 + (lane >> 3);
-        const uint4 raw = *reinterpret_cast<const uint4 *>(codes + r * 128 + c16 * 16);
-        __syncwarp();  // all 4 rows read before any of them is overwritten
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint32_t h[8];
+    constexpr int kRowsPerStep = 16;  // 4 independent 16-byte loads per lane in flight
+#pragma unroll 1
+    for (int step = 0; step < kChunk / kRowsPerStep; ++step) {
+        uint4 raw[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint16_t lo, hi;
-            split_b32(w[j], lo, hi);
-            h[2 * j] = e4m3x2_to_half2_bits(lo);
-            h[2 * j + 1] = e4m3x2_to_half2_bits(hi);
+        for (int k = 0; k < 4; ++k)
+            raw[k] = *reinterpret_cast<const uint4 *>(codes + (step * kRowsPerStep + k * 4 + (lane >> 3)) * 128 +
+                                                      c16 * 16);
+        __syncwarp();  // all 16 rows read before any of them is overwritten
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = step * kRowsPerStep + k * 4 + (lane >> 3);
+            const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+            uint32_t h[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint16_t lo, hi;
+                split_b32(w[j], lo, hi);
+                h[2 * j] = e4m3x2_to_half2_bits(lo);
+                h[2 * j + 1] = e4m3x2_to_half2_bits(hi);
+            }
+            *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
         }
-        *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
         __syncwarp();
     }
 }
