@@ -1,8 +1,8 @@
 /*
  * pa.h -- C ABI of the paged decode attention library (libpa.so, sm_100a).
  *
- * Three operations make one decode step of one attention layer over a KV
- * cache stored in fixed 16-token physical blocks:
+ * The operations of one decode step of one attention layer over a KV cache
+ * stored in fixed 16-token physical blocks, and their variants:
  *
  *   pa_reshape_and_cache  write each new token's key/value into its slot
  *   pa_copy_blocks        copy-on-write duplication of shared blocks
@@ -27,15 +27,19 @@
  * Conventions shared by every call
  * --------------------------------
  * - Every data pointer is a DEVICE pointer on the current CUDA device,
- *   except the two pointer ARRAYS of pa_copy_blocks, which live in host
- *   memory and hold device pointers.  The caller owns every buffer.
+ *   except: the two pointer ARRAYS of pa_copy_blocks (host memory holding
+ *   device pointers); the pools of pa_swap_blocks (device or page-locked
+ *   host memory); and the arrays of pa_prefix_cache_* and pa_prefix_order
+ *   (host memory).  The caller owns every buffer.
  * - The library allocates nothing and never synchronises the stream: work
  *   is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
  *   legacy default stream) and the call returns.
- * - Element type of q, out, caches, key and value: 16-bit, fp16 or bf16
- *   (pa_dims.dtype).  Arithmetic is fp32; outputs round to nearest-even.
+ * - Element type of q, out, key and value: 16-bit, fp16 or bf16
+ *   (pa_dims.dtype); caches hold the same type or FP8 E4M3 codes
+ *   (pa_dims.kv_dtype).  Arithmetic is fp32; outputs round to nearest-even.
  * - Layouts (row-major, contiguous):
- *     q, out         [num_seqs, num_heads, head_dim]
+ *     q, out         [num_seqs, num_heads, head_dim] ([num_seqs, q_len,
+ *                    num_heads, head_dim] for pa_decode_ext)
  *     k/v cache      [num_blocks, num_kv_heads, block_size, head_dim]
  *     block_tables   int32 [num_seqs, max_blocks_per_seq]
  *     context_lens   int32 [num_seqs]
