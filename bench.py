@@ -104,9 +104,19 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# Sources that only the tensor-core kernel is built from: the CUDA-core
+# kernel's traffic does not depend on them.
+TC_ONLY_SOURCES = ("pa_decode_tc.cu", "pa_tc.cuh")
+
+
+def kernel_source_hash(tensor_core: bool = True, root: str = ROOT) -> str:
+    """Hash of the sources a decode kernel is built and launched from: all of
+    csrc/ for the tensor-core kernel, csrc/ without the tensor-core kernel's
+    own files for the CUDA-core kernel."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_424_b200", "csrc", "*"))):
+    for p in sorted(glob.glob(os.path.join(root, "paged_kv_cache_424_b200", "csrc", "*"))):
+        if not tensor_core and os.path.basename(p) in TC_ONLY_SOURCES:
+            continue
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
@@ -121,10 +131,10 @@ def ncu_traffic(workload: str, units: float):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_src_sha") != kernel_source_hash():
-        return None
     ent = rec.get("workloads", {}).get(workload)
     if not ent:
+        return None
+    if ent.get("kernel_src_sha") != kernel_source_hash("decode_tc_kernel" in ent.get("kernel", "")):
         return None
     return float(ent["dram_bytes_per_unit"]) * units
 

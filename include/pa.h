@@ -187,10 +187,15 @@ pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const
  * KV-cache compression as a goal (section 九 item 3).  Same definition as
  * pa_decode with K_s[j] = decode(k code) * k_scale and V_s[j] = decode(v code)
  * * v_scale; q / out in dims->dtype.  Groups of 4, 8 or 16 query heads at
- * head_dim 128 run on the tensor-core kernel (codes widened in shared
- * memory to f16, q converted to f16 for the MMA: a bf16 q must lie within
- * f16's range, |q| <= 65504, and loses precision below 2^-14); other shapes
- * on the CUDA-core kernel.
+ * head_dim 128 run on the tensor-core kernel; other shapes on the CUDA-core
+ * kernel.  With 4 or 8 rows per KV head the tensor cores multiply the E4M3
+ * codes as stored: q is split into three E4M3 parts under a power-of-two
+ * factor per row (q recovered to within 2^-15 of the row's largest |q|, any
+ * finite q) and the softmax weights w into four (|error| <= 2^-12 w +
+ * 2^-22).  With 16 rows (group 16, or several query tokens through
+ * pa_decode_ext) the codes are widened in shared memory to f16 and q is
+ * converted to f16 for the MMA: a bf16 q must then lie within f16's range,
+ * |q| <= 65504, and loses precision below 2^-14.
  * Workspace as from pa_decode_workspace_size with the same dims.
  */
 pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,

@@ -30,8 +30,15 @@
 //           tile, and accumulates O chunk by chunk in registers.
 // Shared memory: K tile 32 KiB + V tile 32 KiB + Q 4 KiB + P 4 KiB (+ <1 KiB)
 // = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
+// FP8 E4M3 caches, groups of 4 or 8: the K and V tiles hold the chunk's
+// codes as loaded (16 KiB each, 128-byte swizzle) and both products run
+// E4M3 x E4M3: S = K . Q^T against Q split into three E4M3 parts (3G
+// columns), O^T = V^T . P^T against P split into four (4G columns); S and
+// O take 4G columns each, 64 or 128 TMEM columns in all.  FP8 with 16
+// columns widens K and V to f16 in place.
 // Results go to `out` (one partition) or to the split workspace for the
 // log-sum-exp merge, exactly like the CUDA-core kernel.
+#include <cfloat>
 #include <climits>
 #include <mutex>
 #include <type_traits>
@@ -60,12 +67,21 @@ constexpr int kRedOff = kPOff + 2 * kN * 128;   // 73728: [2][4][16] floats
 constexpr int kBarOff = kRedOff + 2 * 4 * kN * 4;
 constexpr int kNumBars = 12;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;  // TMEM base, fail flag, 4 lazy-max flags
-constexpr int kSmemTc = kMiscOff + 32;
+constexpr int kQScaleOff = kMiscOff + 32;          // FP8 with E4M3 products: [8] per-row logit factors
+constexpr int kSmemTc = kQScaleOff + 32;
 
-// TMEM columns: S buffers at 0 and 16, O buffers at 32 and 48.
-constexpr uint32_t kTmemCols = 64;
-__device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * kN); }
-__device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)(2 * kN + b * kN); }
+// FP8 caches with groups of 4 or 8 run both products on the E4M3 codes as
+// loaded: Q is split into three E4M3 parts and P into four, stacked as 3G
+// and 4G columns, so S and O have NS = 4G = 16 or 32 columns.  TMEM: S
+// buffers at 0 and NS, O buffers at 2 NS and 3 NS; 64 columns (128 with
+// NS = 32).
+constexpr int kQParts = 3, kPParts = 4;
+__host__ __device__ constexpr int tc_cols(int G, bool e4m3) { return e4m3 && G > 4 ? 32 : kN; }
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int ns) { return 4 * ns <= 64 ? 64u : 128u; }
+template <int NS>
+__device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * NS); }
+template <int NS>
+__device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)(2 * NS + b * NS); }
 
 __device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
 
@@ -91,7 +107,10 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
 // wait until the MMA that read the tile's previous chunk has completed
 // (`empty`), then load the chunk's 8 blocks (zeros past the partition).
 // The table slice is held in registers, 32 entries per window, the next
-// window prefetched one window ahead.
+// window prefetched one window ahead.  kCodes: the tile holds E4M3 codes,
+// one 128-byte row per token (one box per block) instead of two 64-dim
+// regions of 16-bit elements.
+template <bool kCodes = false>
 __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
                                              uint64_t *full, uint64_t *empty, int *fail, int s, int kvh, int b0,
                                              int nb, int nch, int oob_row, int lane) {
@@ -112,13 +131,13 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
         bool ok = true;
         if (lane == 0) {
             ok = c == 0 || wait_ok(empty, (c - 1) & 1, fail);
-            if (ok) mbar_arrive_expect_tx(full, 2 * kRegion);
+            if (ok) mbar_arrive_expect_tx(full, kCodes ? kRegion : 2 * kRegion);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane < kChunkBlocks) {
             tc::tma_load_2d(tile + lane * 2048, tmap, 0, y, full);
-            tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 64, y, full);
+            if constexpr (!kCodes) tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 64, y, full);
         }
     }
 }
@@ -211,9 +230,15 @@ __host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; 
 
 // G: columns of S (query rows per KV head: the group, or group x query
 // tokens with kMasked, padded to a power of two).
-// kFp8: the caches hold E4M3 codes; K, V, Q and P tiles are f16 and the
-// MMA runs f16 x f16 (q converted to f16 on load), k_scale sits in
-// scale_log2 and v_scale multiplies the output.
+// kFp8: the caches hold E4M3 codes; k_scale sits in scale_log2 and v_scale
+// multiplies the output.  With G = 4 or 8 both products run E4M3 x E4M3 on
+// the codes as loaded: Q is split into three E4M3 parts with one
+// power-of-two factor per query row (4 + 4 + 4 significant bits recover a
+// 16-bit q to within 2^-15 of the row's largest |q|), P into four parts
+// (|w - sum| <= 2^-12 w + 2^-22); the f32 products of the parts are
+// recombined when S and O are read from TMEM.  With 16 columns K and V are
+// widened to f16 in place and both products run f16 x f16 (q converted to
+// f16 on load).
 template <typename T, int G, bool kMasked, bool kFp8>
 __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -227,6 +252,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     constexpr int kST = kSW * 32;                // softmax threads
     constexpr int kGT = G > 8 ? 8 : G;           // columns per softmax thread
     constexpr int kWarpK = kSW, kWarpMma = kSW + 1, kWarpV = kSW + 2;
+    constexpr bool kE4m3 = kFp8 && G <= 8;       // both products on the E4M3 codes
+    constexpr int kNS = tc_cols(G, kE4m3);       // columns of S and O
+    constexpr uint32_t kTmemCols = tc_tmem_cols(kNS);
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *k_t = smem + kKOff;
     unsigned char *v_t = smem + kVOff;
@@ -237,6 +265,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     uint64_t *k_full = bars + 0, *k_empty = bars + 1, *v_full = bars + 2, *v_empty = bars + 3;
     uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8, *q_full = bars + 9;
     uint64_t *k_stage = bars + 10, *v_stage = bars + 11;  // FP8: codes landed
+    float *qscale = reinterpret_cast<float *>(smem + kQScaleOff);  // kE4m3: logit factor per query row
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMiscOff);
     int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
     int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
@@ -291,9 +320,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     if (tid == 0) {
         *fail = 0;
         for (int i = 0; i < 4; ++i) lazy_flag[i] = 0;
-        mbar_init(k_full, kFp8 ? 32 : 1);  // FP8: the producer's 32 lanes after converting
+        mbar_init(k_full, kFp8 && !kE4m3 ? 32 : 1);  // widened in place: the producer's 32 lanes
         mbar_init(k_empty, 1);
-        mbar_init(v_full, kFp8 ? 32 : 1);
+        mbar_init(v_full, kFp8 && !kE4m3 ? 32 : 1);
         mbar_init(v_empty, 1);
         mbar_init(k_stage, 1);
         mbar_init(v_stage, 1);
@@ -311,29 +340,46 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpK) {
-        if constexpr (kFp8)
+        if constexpr (kE4m3)
+            produce_tile<true>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        else if constexpr (kFp8)
             produce_tile_fp8(p, &tmap_k, k_t, k_stage, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
         else
             produce_tile(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
     } else if (warp == kWarpV) {
-        if constexpr (kFp8)
+        if constexpr (kE4m3)
+            produce_tile<true>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        else if constexpr (kFp8)
             produce_tile_fp8(p, &tmap_v, v_t, v_stage, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
         else
             produce_tile(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = tc::instr_desc_f16(kBf16, false, kChunk, kN);
-            constexpr uint32_t idesc_pv = tc::instr_desc_f16(kBf16, true, kD, kN);
+            constexpr uint32_t idesc_qk =
+                kE4m3 ? tc::instr_desc_e4m3(false, kChunk, kNS) : tc::instr_desc_f16(kBf16, false, kChunk, kN);
+            constexpr uint32_t idesc_pv =
+                kE4m3 ? tc::instr_desc_e4m3(true, kD, kNS) : tc::instr_desc_f16(kBf16, true, kD, kN);
             const uint32_t kb = smem_addr(k_t), vb = smem_addr(v_t), qb = smem_addr(q_t), pb = smem_addr(p_t);
             auto pv = [&](int c) -> bool {
                 if (!wait_ok(p_full, c & 1, fail) || !wait_ok(v_full, c & 1, fail)) return false;
                 tc::fence_after_sync();
+                if constexpr (kE4m3) {
+                    // V codes MN-major (a token's 128 dims are one 128-byte atom row),
+                    // 32 tokens per MMA; P parts K-major, one 128-byte row per column
 #pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk) {
-                    const uint64_t a = tc::smem_desc(vb + kk * 2048, kRegion, 1024);
-                    const uint64_t b = tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-                    tc::mma_f16(tmem + o_col(c & 1), a, b, idesc_pv, kk > 0);
+                    for (int kk = 0; kk < kChunk / 32; ++kk) {
+                        const uint64_t a = tc::smem_desc(vb + kk * 4096, kRegion, 1024);
+                        const uint64_t b = tc::smem_desc(pb + kk * 32, 16, 1024);
+                        tc::mma_e4m3(tmem + o_col<kNS>(c & 1), a, b, idesc_pv, kk > 0);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kChunk / 16; ++kk) {
+                        const uint64_t a = tc::smem_desc(vb + kk * 2048, kRegion, 1024);
+                        const uint64_t b = tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+                        tc::mma_f16(tmem + o_col<kNS>(c & 1), a, b, idesc_pv, kk > 0);
+                    }
                 }
                 tc::commit(&o_full[c & 1]);
                 tc::commit(v_empty);
@@ -344,11 +390,21 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 ok = wait_ok(k_full, c & 1, fail);
                 if (!ok) break;
                 tc::fence_after_sync();
+                if constexpr (kE4m3) {
+                    // K codes: one 128-byte row per token; Q parts: one 128-byte row per column
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t a = tc::smem_desc(kb + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = tc::smem_desc(qb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-                    tc::mma_f16(tmem + s_col(c & 1), a, b, idesc_qk, kk > 0);
+                    for (int kk = 0; kk < kD / 32; ++kk) {
+                        const uint64_t a = tc::smem_desc(kb + kk * 32, 16, 1024);
+                        const uint64_t b = tc::smem_desc(qb + kk * 32, 16, 1024);
+                        tc::mma_e4m3(tmem + s_col<kNS>(c & 1), a, b, idesc_qk, kk > 0);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint64_t a = tc::smem_desc(kb + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
+                        const uint64_t b = tc::smem_desc(qb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+                        tc::mma_f16(tmem + s_col<kNS>(c & 1), a, b, idesc_qk, kk > 0);
+                    }
                 }
                 tc::commit(&s_full[c & 1]);
                 tc::commit(k_empty);
@@ -364,6 +420,51 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             // K-major 128-byte swizzle, two 64-dim regions.  Loaded while the
             // producers already stream K and V.
             const T *q = reinterpret_cast<const T *>(p.q);
+            if constexpr (kE4m3) {
+                // Q as E4M3 parts, one warp per query row r, lane l holding
+                // dims 4l .. 4l + 3: y = q * 2^e with max |y| in [128, 256),
+                // hi = E4M3(y), mid = E4M3(16 (y - hi)), lo = E4M3(16 (16 (y - hi) - mid)),
+                // so q = 2^-e (hi + mid / 16 + lo / 256) + err, |err| <= 2^-15 max |q|.
+                // Rows hi: r, mid: G + r, lo: 2G + r of the 128-byte-swizzled
+                // tile; padding rows zero.  qscale[r] = scale_log2 * 2^-e.
+                for (int r = warp; r < G; r += kSW) {
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (r < rows) {
+                        const uint2 raw = *reinterpret_cast<const uint2 *>(q + row_of(r) * kD + 4 * lane);
+                        const float2 a = E::to_float2(raw.x), b = E::to_float2(raw.y);
+                        y[0] = a.x;
+                        y[1] = a.y;
+                        y[2] = b.x;
+                        y[3] = b.y;
+                    }
+                    float mx = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    const bool finite = mx <= FLT_MAX;  // false for inf and NaN
+                    int e = 0;
+                    if (mx > 0.f && finite) {
+                        int k;
+                        (void)frexpf(mx, &k);  // mx in [2^(k-1), 2^k)
+                        e = 8 - k;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) y[i] = ldexpf(y[i], e);
+#pragma unroll
+                    for (int part = 0; part < kQParts; ++part) {
+                        const uint16_t c01 = float2_to_e4m3x2(y[0], y[1]), c23 = float2_to_e4m3x2(y[2], y[3]);
+                        *reinterpret_cast<uint32_t *>(q_t + tc::sw128_offset8(part * G + r, 4 * lane)) =
+                            (uint32_t)c01 | ((uint32_t)c23 << 16);
+                        const float2 d01 = e4m3x2_to_float2(c01), d23 = e4m3x2_to_float2(c23);
+                        y[0] = (y[0] - d01.x) * 16.f;  // exact: the rounding error of y
+                        y[1] = (y[1] - d01.y) * 16.f;
+                        y[2] = (y[2] - d23.x) * 16.f;
+                        y[3] = (y[3] - d23.y) * 16.f;
+                    }
+                    if (lane == 0) qscale[r] = finite ? ldexpf(p.scale_log2, -e) : NAN;
+                }
+                for (int r = kQParts * G + warp; r < kNS; r += kSW)  // padding columns
+                    *reinterpret_cast<uint32_t *>(q_t + tc::sw128_offset8(r, 4 * lane)) = 0u;
+            } else {
             for (int i = tid; i < kN * (kD / 8); i += kST) {
                 const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
                 uint4 v = make_uint4(0, 0, 0, 0);
@@ -381,8 +482,10 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 }
                 *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
             }
+            }
             fence_proxy_async_smem();
             mbar_arrive(q_full);
+            if constexpr (kE4m3) softmax_sync<kST>();  // qscale written by every softmax warp
         }
         const int t = tid & 127;                                      // token of S, dim of O
         const int c0 = kSW == 8 ? (warp >> 2) * kGT : 0;              // this thread's first column
@@ -393,6 +496,30 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
         const int hi0 = L - p.q_len;
         const int lg = 31 - __clz(p.group);
         const int win = p.window > 0 ? p.window : INT_MAX;
+        // E4M3 products: column j of the result = sum over parts k of part
+        // column kG + j / 16^k (Horner from the last part) of the TMEM buffer at taddr
+        auto ld_parts = [&](auto np, uint32_t taddr, float *v) {
+            constexpr int NP = decltype(np)::value;
+            if constexpr (G == 4) {
+                float t16[16];
+                tc::tmem_ld<16>(taddr, t16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float a = t16[(NP - 1) * 4 + j];
+#pragma unroll
+                    for (int k = NP - 2; k >= 0; --k) a = fmaf(a, 0.0625f, t16[k * 4 + j]);
+                    v[j] = a;
+                }
+            } else {
+                float b[8];
+#pragma unroll
+                for (int k = NP - 1; k >= 0; --k) {
+                    tc::tmem_ld<8>(taddr + 8 * k, b);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = k == NP - 1 ? b[j] : fmaf(v[j], 0.0625f, b[j]);
+                }
+            }
+        };
         // per-thread state of columns c0 + j, j < kGT
         float m[kGT], l[kGT], acc[kGT], alpha_prev[kGT];
 #pragma unroll
@@ -406,7 +533,10 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             if (!wait_ok(&o_full[c & 1], (c >> 1) & 1, fail)) return;
             tc::fence_after_sync();
             float o[8];
-            tc::tmem_ld<8>(tmem + lane_base + o_col(c & 1) + c0, o);
+            if constexpr (kE4m3)
+                ld_parts(std::integral_constant<int, kPParts>{}, tmem + lane_base + o_col<kNS>(c & 1), o);
+            else
+                tc::tmem_ld<8>(tmem + lane_base + o_col<kNS>(c & 1) + c0, o);
 #pragma unroll
             for (int j = 0; j < kGT; ++j) acc[j] = fmaf(acc[j], alpha_prev[j], o[j]);
         };
@@ -479,7 +609,17 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             if (ok) {
                 tc::fence_after_sync();
                 float sv[8];
-                tc::tmem_ld<8>(tmem + lane_base + s_col(c & 1) + c0, sv);
+                const uint32_t sb = tmem + lane_base + s_col<kNS>(c & 1);
+                float scl[kGT];
+                if constexpr (kE4m3) {
+                    ld_parts(std::integral_constant<int, kQParts>{}, sb, sv);
+#pragma unroll
+                    for (int j = 0; j < kGT; ++j) scl[j] = qscale[j];
+                } else {
+                    tc::tmem_ld<8>(sb + c0, sv);
+#pragma unroll
+                    for (int j = 0; j < kGT; ++j) scl[j] = p.scale_log2;
+                }
 #pragma unroll
                 for (int j = 0; j < kGT; ++j) {
                     bool live = valid;
@@ -488,7 +628,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                         const int pos = hi0 + (h >> lg);
                         live = live && h < rows && tok <= pos && pos - tok < win;
                     }
-                    x[j] = live ? sv[j] * p.scale_log2 : -INFINITY;
+                    x[j] = live ? sv[j] * scl[j] : -INFINITY;
                     exceed |= x[j] > m[j] + kLazyMax;
                 }
             } else {
@@ -527,11 +667,38 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 }
             }
             MT pv[kGT];
+            uint16_t pc[kPParts][kGT / 2];  // E4M3: the weights' parts, two columns per code pair
+            if constexpr (kE4m3) {
+                // w = sum over k of part_k / 16^k, part_0 = E4M3(w), part_k = E4M3(16 r_k) with
+                // r_k the remainder after part k - 1; w <= 2^8 (the lazy max), so no part
+                // saturates, and |w - sum| <= 2^-12 w + 2^-22
 #pragma unroll
-            for (int j = 0; j < kGT; ++j) {
-                // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
-                pv[j] = (kMasked && x[j] == -INFINITY) ? EM::from_float(0.f) : EM::from_float(ex2(x[j] - m[j]));
-                l[j] += EM::to_float(pv[j]);  // the rounded weight the MMA sees
+                for (int j = 0; j < kGT; j += 2) {
+                    // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
+                    float a = x[j] == -INFINITY ? 0.f : ex2(x[j] - m[j]);
+                    float b = x[j + 1] == -INFINITY ? 0.f : ex2(x[j + 1] - m[j + 1]);
+                    float wa = 0.f, wb = 0.f, f = 1.f;
+#pragma unroll
+                    for (int k = 0; k < kPParts; ++k) {
+                        const uint16_t cc = float2_to_e4m3x2(a, b);
+                        const float2 d = e4m3x2_to_float2(cc);
+                        pc[k][j / 2] = cc;
+                        wa = fmaf(d.x, f, wa);
+                        wb = fmaf(d.y, f, wb);
+                        a = (a - d.x) * 16.f;
+                        b = (b - d.y) * 16.f;
+                        f *= 0.0625f;
+                    }
+                    l[j] += wa;  // the weight the MMA sees (to f32 rounding)
+                    l[j + 1] += wb;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kGT; ++j) {
+                    // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
+                    pv[j] = (kMasked && x[j] == -INFINITY) ? EM::from_float(0.f) : EM::from_float(ex2(x[j] - m[j]));
+                    l[j] += EM::to_float(pv[j]);  // the rounded weight the MMA sees
+                }
             }
             if (cl > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
 #pragma unroll
@@ -542,7 +709,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 // once it has landed, so 0 * V stays 0 in the PV product.
                 if (wait_ok(v_full, c & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
+                    for (int j = 0; j < (kE4m3 ? 1 : 2); ++j)  // E4M3: a token's codes are one 128-byte row
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             *reinterpret_cast<uint4 *>(v_t + j * kRegion + t * 128 + k * 16) = make_uint4(0, 0, 0, 0);
@@ -551,12 +718,22 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             // P tile: K-major, rows = heads, columns = tokens (two 64-token
             // regions); this thread writes rows c0 .. c0 + (16 / (kSW / 4)) - 1
             // (its columns, then zero rows up to 16)
-            unsigned char *pr = p_t + (t >> 6) * (kN * 128);
-            constexpr int kRowsW = kN / (kSW / 4);
+            if constexpr (kE4m3) {
+                // E4M3 part tile: part k of column j in row k G + j, one 128-byte
+                // row of tokens each
 #pragma unroll
-            for (int j = 0; j < kRowsW; ++j) {
-                const MT v = j < kGT ? pv[j < kGT ? j : 0] : EM::from_float(0.f);
-                *reinterpret_cast<MT *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
+                for (int k = 0; k < kPParts; ++k)
+#pragma unroll
+                    for (int j = 0; j < kGT; ++j)
+                        p_t[tc::sw128_offset8(k * G + j, t)] = (unsigned char)(pc[k][j / 2] >> (8 * (j & 1)));
+            } else {
+                unsigned char *pr = p_t + (t >> 6) * (kN * 128);
+                constexpr int kRowsW = kN / (kSW / 4);
+#pragma unroll
+                for (int j = 0; j < kRowsW; ++j) {
+                    const MT v = j < kGT ? pv[j < kGT ? j : 0] : EM::from_float(0.f);
+                    *reinterpret_cast<MT *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
+                }
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
@@ -595,8 +772,9 @@ EncodeTiledFn encode_fn() {
 // A cache [NB, Hk, 16, 128] seen as rows of 128 elements; boxes of 16 rows
 // x 64 elements with the 128-byte swizzle; out-of-range rows read as zero.
 // An FP8 cache [NB, Hk, 16, 128] seen as rows of 128 one-byte codes; boxes
-// of 16 rows x 128 bytes, unswizzled (the producer converts them).
-bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows) {
+// of 16 rows x 128 bytes, unswizzled where the producer converts them,
+// with the 128-byte swizzle where the MMA reads them.
+bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows, bool swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
@@ -604,7 +782,8 @@ bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows) {
     const cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kBlock};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -625,7 +804,7 @@ template <typename T, int G, bool kMasked, bool kFp8 = false>
 cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
     CUtensorMap tk, tv;
-    const bool ok = kFp8 ? encode_code_map(&tk, p.k_cache, rows) && encode_code_map(&tv, p.v_cache, rows)
+    const bool ok = kFp8 ? encode_code_map(&tk, p.k_cache, rows, G <= 8) && encode_code_map(&tv, p.v_cache, rows, G <= 8)
                          : encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) &&
                                encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value);
     if (!ok) return cudaErrorInvalidValue;

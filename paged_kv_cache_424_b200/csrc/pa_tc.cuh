@@ -19,10 +19,13 @@
 //   MN-major operand (the 64 M/N-elements of an atom row contiguous, rows =
 //   K): LBO = byte distance between 64-element M/N atoms, SBO = byte
 //   distance between 8-row K groups.
-// Instruction descriptor (kind::f16): bits 4-5 D format (1 = f32), 7-9 A
-// format and 10-12 B format (0 = f16, 1 = bf16; A and B always the same
-// type here), bit 15 / 16 A / B major (0 = K, 1 = MN), bits 17-22 N >> 3,
-// bits 24-28 M >> 4.
+// With one-byte elements (E4M3) an atom row holds 128 elements.
+// Instruction descriptor (kind::f16 and kind::f8f6f4): bits 4-5 D format
+// (1 = f32), 7-9 A format and 10-12 B format (kind::f16: 0 = f16, 1 = bf16;
+// kind::f8f6f4: 0 = E4M3; A and B always the same type here), bit 15 / 16
+// A / B major (0 = K, 1 = MN), bits 17-22 N >> 3, bits 24-28 M >> 4.
+// One kind::f16 MMA takes K = 16 elements, one kind::f8f6f4 MMA K = 32: 32
+// bytes of each K-major row either way.
 #pragma once
 
 #include <cuda.h>
@@ -47,6 +50,11 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(bool bf16, bool a_mn_major
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// E4M3 x E4M3 -> f32; B K-major, A K-major or MN-major.
+__host__ __device__ constexpr uint32_t instr_desc_e4m3(bool a_mn_major, int M, int N) {
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] * B[smem], issued by one thread.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         bool accumulate) {
@@ -54,6 +62,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// The same for E4M3 operands (kind::f8f6f4).
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
 }
@@ -130,6 +149,11 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tmap, 
 // region whose rows are 128 bytes (64 16-bit elements).
 __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 3) ^ row) & 7) << 4) + (col & 7) * 2);
+}
+
+// The same for a tile of one-byte elements (rows of 128 elements).
+__device__ __forceinline__ uint32_t sw128_offset8(int row, int col) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 4) ^ row) & 7) << 4) + (col & 15));
 }
 
 }  // namespace tc
