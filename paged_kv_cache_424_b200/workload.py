@@ -310,7 +310,7 @@ def gqa8b(seed: int = 2, num_seqs: int = 256, num_steps: int = 1, churn: float =
     step retires round(churn * S) of them (chosen by the seeded RNG), admits
     as many new ones and appends one token to every survivor."""
     rng = np.random.default_rng(seed)
-    mb = -(-(cap + num_steps) // BLOCK_SIZE)
+    mb = -(-(max(cap, new_max) + num_steps) // BLOCK_SIZE)  # admitted sequences grow too
     dims = Dims(num_seqs, 32, 8, 128, BLOCK_SIZE, mb, num_blocks, "bf16")
     b = _Builder(rng, dims, v_lo=v_lo)
     b.admit_pad()
