@@ -5,14 +5,24 @@ A step is one pass of the whole hot path over one batch: the cache write of
 every sequence's new token (pa_reshape_and_cache), copy-on-write copies when
 the workload has them (pa_copy_blocks), and decode attention of every
 sequence over its paged KV cache (pa_decode, with the split-KV merge when a
-context spans several 512-token partitions).  Default workload: the
-Llama-2-7B-shaped MHA batch (64 sequences, lengths U[128, 2048], 32 heads,
-head_dim 128, fp16, 16384-block pool).
+context spans several partitions).
+
+Default workload: the Llama-3-8B-shaped GQA batch under continuous batching
+(256 sequences, lognormal lengths with median 1024 capped at 4096, 32 query
+heads over 8 KV heads, head_dim 128, bf16, 131072-block pool).  Every step
+retires 26 sequences and admits 26 new ones of 32-512 tokens; the rest grow
+by one token.  The scenario is built with two set-up steps followed by a
+cycle of --cycle churned steps (8 by default), all of whose inputs are on
+the device before timing; the timed loop walks through the cycle, so
+consecutive timed steps decode different batch mixes.  The same JSON line
+carries `config.also`: the decode time and roofline fraction of the
+long-context 70B shape at its stated 512-token partitions, the
+copy-on-write batch and the 7B MHA batch, measured in the same run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--kv 16|fp8]
   python bench.py --impl reference ...      # the CPU oracle, timed the same way
 
-Other workloads: gqa8b, long70b, cow (the pages' other shapes), spec8b (4
+Other workloads: mha7b, long70b, cow (the pages' other shapes), spec8b (4
 query tokens per sequence, pa_decode_ext), window70b (4096-token sliding
 window), prefix8b (shared prefixes in a shuffled batch, decoded in the
 pa_prefix_order schedule; the batch-order time is reported beside), swap
@@ -43,7 +53,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention seqs/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
+TARGET_GBS = 8000.0  # the HBM peak the 70 % target is stated against
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+WORKLOADS = ["tiny", "mha7b", "gqa8b", "long70b", "cow", "spec8b", "window70b", "prefix8b", "swap"]
+DEFAULT_ALSO = "long70b,cow,mha7b,gqa8b:fp8,long70b:fp8"
 
 
 # ---------------------------------------------------------------------------
@@ -55,11 +68,16 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha7b",
-                    choices=["tiny", "mha7b", "gqa8b", "long70b", "cow", "spec8b", "window70b", "prefix8b", "swap"],
+    ap.add_argument("--workload", default="gqa8b", choices=WORKLOADS,
                     help="decode scenario (spec8b: 4 query tokens per sequence; window70b: 4096-token sliding "
                          "window; prefix8b: shuffled batch of shared 2000-token prefixes, decoded in "
                          "shared-prefix order), or 'swap' for pa_swap_blocks device <-> pinned host throughput")
+    ap.add_argument("--cycle", type=int, default=8,
+                    help="gqa8b: churned steps in the timed cycle (after two set-up steps)")
+    ap.add_argument("--also", default=None,
+                    help=f"comma-separated workloads whose decode is measured after the main one and reported "
+                         f"in config.also (default for gqa8b: {DEFAULT_ALSO}; 'none' for none; a name may end "
+                         f"in ':fp8' for an FP8 cache)")
     ap.add_argument("--num-seqs", type=int, default=None, help="override the batch size (profiling cases)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override the pool size (profiling cases)")
     ap.add_argument("--partition", type=int, default=None, help="partition tokens (default: the workload's)")
@@ -73,13 +91,13 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def make_scenario(name: str, seed: int, num_seqs=None, num_blocks=None, kv: str = "16"):
+def make_scenario(name: str, seed: int, num_seqs=None, num_blocks=None, kv: str = "16", cycle: int = 8):
     from paged_kv_cache_424_b200 import workload as W
-    sc = _base_scenario(name, seed, num_seqs, num_blocks)
+    sc = _base_scenario(name, seed, num_seqs, num_blocks, cycle)
     return W.with_fp8_cache(sc) if kv == "fp8" else sc
 
 
-def _base_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
+def _base_scenario(name: str, seed: int, num_seqs=None, num_blocks=None, cycle: int = 8):
     from paged_kv_cache_424_b200 import workload as W
     kw = {}
     if num_seqs is not None:
@@ -88,11 +106,22 @@ def _base_scenario(name: str, seed: int, num_seqs=None, num_blocks=None):
         kw["num_blocks"] = num_blocks
     if name == "tiny":
         return W.tiny(seed)
+    if name == "gqa8b":
+        return W.gqa8b(seed, num_steps=2 + max(1, cycle), **kw)
     if name in ("cow", "prefix8b"):
         if num_seqs is not None:
             kw = {"num_prompts": max(1, num_seqs // 8), **({"num_blocks": num_blocks} if num_blocks else {})}
         return getattr(W, name)(seed, **kw)
     return getattr(W, name)(seed, **kw)
+
+
+def scenario_cycle(sc):
+    """(set-up steps, timed cycle).  A continuous-batching scenario with
+    churned steps keeps its first two steps as set-up and times the rest in
+    turn; a one-step scenario times its one step over and over."""
+    if len(sc.steps) > 2:
+        return sc.steps[:2], sc.steps[2:]
+    return sc.steps[:-1], sc.steps[-1:]
 
 
 def measured_hbm_peak():
@@ -163,17 +192,21 @@ class ClockSampler:
             self.nv = None
             self.err = str(e)
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
         if self.nv is not None:
+            self._sample()  # at least one sample inside the region, however short
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
@@ -219,19 +252,283 @@ def barrier(world: int):
         dist.barrier()
 
 
+def also_list(args):
+    spec = args.also if args.also is not None else (DEFAULT_ALSO if args.workload == "gqa8b" else "none")
+    if spec.strip().lower() in ("", "none"):
+        return []
+    out = []
+    for item in spec.split(","):
+        name, _, kv = item.strip().partition(":")
+        if name not in WORKLOADS or name == "swap":
+            raise SystemExit(f"--also: unknown workload {name!r}")
+        out.append((name, "fp8" if kv == "fp8" else "16"))
+    return out
+
+
 # ---------------------------------------------------------------------------
-# our arm
+# our arm: one workload on the device
 # ---------------------------------------------------------------------------
+class DeviceWorkload:
+    """A scenario resident on the device: every cache operation of every
+    step applied (admissions, copies, writes), and for each step of the timed
+    cycle its decode inputs, new tokens, slots and copy pairs on the device,
+    so that a timed step enqueues only the library's kernels."""
+
+    def __init__(self, sc, device, partition, pa, W):
+        import torch
+        from paged_kv_cache_424_b200.session import DeviceSession
+        self.sc, self.pa, self.W, self.torch = sc, pa, W, torch
+        self.device = device
+        self.fp8 = sc.kv_dtype == "fp8"
+        self.P = sc.partition_tokens if partition is None else partition
+        self.dev = DeviceSession(sc, device=str(device))
+        setup, cycle = scenario_cycle(sc)
+        for st in setup + cycle:
+            self.dev.apply_cache_ops(st)
+        self.items = []
+        for st in cycle:
+            inp = self.dev.decode_inputs(st)
+            writes = self.dev.write_inputs(st)
+            bm = torch.from_numpy(np.ascontiguousarray(st.block_mapping)).to(device) if st.block_mapping.size \
+                else None
+            maxlen = st.max_context_len
+            if sc.ext:
+                ws_bytes = self.dev.ext_workspace_bytes(inp, maxlen, self.P)
+                nparts = None
+            else:
+                dims = pa.dims_of(inp["q"], self.dev.k_cache, inp["block_tables"])
+                nparts = pa.pa_decode_num_partitions(dims, maxlen, self.P)
+                ws_bytes = pa.pa_decode_workspace_size(dims, maxlen, self.P)
+            kv_logical = W.kv_bytes(st, sc.dims, elem_bytes=sc.kv_elem_bytes, q_len=sc.q_len, window=sc.window)
+            kv = (W.kv_bytes(st, sc.dims, unique=True, elem_bytes=sc.kv_elem_bytes)
+                  if sc.name.split("-")[0] in ("cow", "prefix8b") else kv_logical)
+            qo = W.qo_bytes(sc.dims, sc.q_len)
+            launches = (1 if bm is not None else 0) + len(writes) + (2 if ws_bytes else 1)
+            self.items.append(dict(step=st, inp=inp, writes=writes, bm=bm, maxlen=maxlen, ws_bytes=ws_bytes,
+                                   nparts=nparts, kv=kv, kv_logical=kv_logical, algo=kv + qo,
+                                   logical=kv_logical + qo, launches=launches))
+        self.ws = self.dev.workspace(max(it["ws_bytes"] for it in self.items))
+        self.out = torch.empty_like(self.items[0]["inp"]["q"])
+
+    # -- the library calls of one step -----------------------------------------
+    def write(self, key, value, slots, stream):
+        sc, pa, dev = self.sc, self.pa, self.dev
+        if self.fp8:
+            pa.pa_reshape_and_cache_fp8(key, value, dev.k_cache, dev.v_cache, slots, sc.k_scale, sc.v_scale,
+                                        stream=stream)
+        else:
+            pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
+
+    def decode(self, it, q, bt, cl, out, stream, seq_order=None):
+        sc, pa, dev = self.sc, self.pa, self.dev
+        if sc.ext:
+            dev.decode_ext({"q": q, "block_tables": bt, "context_lens": cl, "seq_order": seq_order}, it["maxlen"],
+                           self.P, out, stream=stream)
+        elif self.fp8:
+            pa.pa_decode_fp8(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.k_scale, sc.v_scale,
+                             sc.dims.num_kv_heads, it["maxlen"], self.P, self.ws, stream=stream)
+        else:
+            pa.pa_decode(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.dims.num_kv_heads, it["maxlen"],
+                         self.P, self.ws, stream=stream)
+
+    def step(self, it, stream, e0=None, e1=None, seq_order="default"):
+        pa, dev = self.pa, self.dev
+        if it["bm"] is not None:
+            pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], it["bm"], stream=stream)
+        for key, value, slots in it["writes"]:
+            self.write(key, value, slots, stream)
+        if e0 is not None:
+            e0.record(stream)
+        inp = it["inp"]
+        so = inp.get("seq_order") if seq_order == "default" else seq_order
+        self.decode(it, inp["q"], inp["block_tables"], inp["context_lens"], self.out, stream, so)
+        if e1 is not None:
+            e1.record(stream)
+
+    # -- timing ----------------------------------------------------------------
+    def time_steps(self, K, warmup, stream, world, seq_order="default", clocks=None):
+        """Two timed loops of K steps over the cycle, after `warmup` untimed
+        ones.  The step loop has events only at its two ends, so consecutive
+        kernels keep their programmatic-dependent-launch overlap: total ms
+        (max over ranks).  The kernel loop repeats the same steps with an
+        event pair around every decode launch: per-launch decode ms (this
+        rank) and the cycle item of each."""
+        torch = self.torch
+        C = len(self.items)
+        for i in range(warmup):
+            self.step(self.items[i % C], stream, seq_order=seq_order)
+        torch.cuda.synchronize(self.device)
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(self.device)
+        ctx = clocks if clocks is not None else _NullCtx()
+        with ctx:
+            start.record(stream)
+            for i in range(K):
+                self.step(self.items[(warmup + i) % C], stream, seq_order=seq_order)
+            end.record(stream)
+            torch.cuda.synchronize(self.device)
+            barrier(world)
+            for i in range(K):
+                self.step(self.items[(warmup + i) % C], stream, e0[i], e1[i], seq_order=seq_order)
+            torch.cuda.synchronize(self.device)
+        barrier(world)
+        ms_total = max_over_ranks(start.elapsed_time(end), world, self.device)
+        dec_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
+        idx = [(warmup + i) % C for i in range(K)]
+        return ms_total, dec_ms, idx
+
+    def roofline_of(self, dec_ms, idx, world):
+        """Algorithmic bytes of the timed decodes over their summed time."""
+        algo = sum(self.items[j]["algo"] for j in idx)
+        logical = sum(self.items[j]["logical"] for j in idx)
+        t = max_over_ranks(sum(dec_ms), world, self.device) / 1e3
+        return algo / t / 1e9, logical / t / 1e9, algo / len(idx), t / len(idx) * 1e3
+
+    # -- end to end ------------------------------------------------------------
+    def e2e(self, K, warmup, stream, world):
+        """The same steps through the same calls with their inputs in pinned
+        host memory: per step, one host-to-device copy of all the step's
+        inputs (query, tables, lengths, new keys / values / slots, copy
+        pairs, schedule) packed in one buffer, the step's kernels reading
+        them in place, and one device-to-host copy of the output.  Copies run
+        on their own streams, double-buffered and ordered by events, so the
+        upload of step i + 1 and the download of step i - 1 overlap step i."""
+        torch, pa = self.torch, self.pa
+        dev = self.device
+        C = len(self.items)
+        packs = [self._pack(it) for it in self.items]
+        nbytes = max(p["nbytes"] for p in packs)
+        staging = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        views = [[self._views(p, staging[b]) for b in range(2)] for p in packs]
+        outs = [torch.empty_like(self.out) for _ in range(2)]
+        h_out = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory() for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        ev_host = [torch.cuda.Event() for _ in range(C)]  # last upload that read host pack j
+        host_order = self.sc.prefix_order
+
+        def run(i):
+            b, j = i % 2, i % C
+            p, v = packs[j], views[j][b]
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev_done[b])  # staging b: step i - 2 has finished with it
+                if host_order:
+                    ev_host[j].synchronize()      # the host pack is free again
+                    p["arrays"]["seq_order"][:] = pa.pa_prefix_order(p["arrays"]["block_tables"],
+                                                                     p["arrays"]["context_lens"])
+                staging[b].copy_(p["host"], non_blocking=True)
+                ev_in[b].record(h2d_s)
+                ev_host[j].record(h2d_s)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])      # outs[b]: step i - 2's output has been read back
+            it = self.items[j]
+            if "bm" in v:
+                pa.pa_copy_blocks([self.dev.k_cache], [self.dev.v_cache], v["bm"], stream=stream)
+            for w in range(len(it["writes"])):
+                self.write(v[f"key{w}"], v[f"value{w}"], v[f"slots{w}"], stream)
+            self.decode(it, v["q"], v["block_tables"], v["context_lens"], outs[b], stream, v.get("seq_order"))
+            ev_done[b].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[b])
+                h_out[b].copy_(outs[b], non_blocking=True)
+                ev_out[b].record(d2h_s)
+
+        for i in range(warmup):
+            run(i)
+        torch.cuda.synchronize(dev)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        h2d_s.wait_event(a)
+        for i in range(warmup, warmup + K):
+            run(i)
+        stream.wait_event(ev_out[(warmup + K - 1) % 2])
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ms = max_over_ranks(a.elapsed_time(z), world, dev)
+        h2d = sum(packs[(warmup + i) % C]["nbytes"] for i in range(K)) / K
+        d2h = self.out.numel() * self.out.element_size()
+        return {"value": self.sc.dims.num_seqs * K * world / (ms / 1e3), "unit": "seqs/s",
+                "h2d_bytes_per_step": int(round(h2d)), "d2h_bytes_per_step": int(d2h), "steps": K,
+                "ms_per_step": ms / K,
+                "path": "pinned host pack -> one cudaMemcpyAsync (copy stream) -> pa_* C-ABI calls reading the "
+                        "device pack -> one cudaMemcpyAsync of the output back (second copy stream); "
+                        "double-buffered, event-ordered"}
+
+    def _pack(self, it):
+        """The step's host inputs laid out in one pinned buffer (256-byte
+        aligned pieces)."""
+        torch = self.torch
+        st = it["step"]
+        pieces = {"q": np.ascontiguousarray(st.q).view(np.uint16),
+                  "block_tables": np.ascontiguousarray(st.block_tables, dtype=np.int32),
+                  "context_lens": np.ascontiguousarray(st.context_lens, dtype=np.int32)}
+        for w, wr in enumerate(st.writes):
+            pieces[f"key{w}"] = np.ascontiguousarray(wr.key)
+            pieces[f"value{w}"] = np.ascontiguousarray(wr.value)
+            pieces[f"slots{w}"] = np.ascontiguousarray(wr.slot_mapping, dtype=np.int64)
+        if st.block_mapping.size:
+            pieces["bm"] = np.ascontiguousarray(st.block_mapping, dtype=np.int64)
+        if self.sc.prefix_order:
+            pieces["seq_order"] = np.zeros(st.context_lens.shape, np.int32)
+        layout, off = {}, 0
+        for k, a in pieces.items():
+            layout[k] = (off, a.dtype, a.shape, a.nbytes)
+            off += (a.nbytes + 255) // 256 * 256
+        host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        hb = host.numpy()
+        arrays = {}
+        for k, a in pieces.items():
+            o, dt, shape, n = layout[k]
+            hb[o:o + n] = a.view(np.uint8).ravel()
+            arrays[k] = hb[o:o + n].view(dt).reshape(shape)
+        return {"host": host, "layout": layout, "nbytes": off, "arrays": arrays}
+
+    def _views(self, p, buf):
+        torch = self.torch
+        tdt = {"q": self.dev.dtype}
+        for k in p["layout"]:
+            if k.startswith("key") or k.startswith("value"):
+                tdt[k] = self.dev.dtype
+        npt = {np.dtype(np.int32): torch.int32, np.dtype(np.int64): torch.int64}
+        out = {}
+        for k, (o, dt, shape, n) in p["layout"].items():
+            t = buf[o:o + n]
+            t = t.view(tdt[k]) if k in tdt else t.view(npt[np.dtype(dt)])
+            out[k] = t.view(shape)
+        return out
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
 def cpu_baseline(sc, seconds: float):
-    """The oracle as it stands on this host's cores, on repeated full steps of
-    the workload (or a subset of its sequences when one step is too long)."""
+    """The oracle as it stands on this host's cores, on the first step of the
+    timed cycle (the cache write of the step plus decode of as many of its
+    sequences as fit the time budget, repeated)."""
     import oracle
     from oracle.harness import OracleSession
     orc = oracle.load()
     cores = orc.max_threads()
-    st = sc.steps[0]
+    setup, cycle = scenario_cycle(sc)
+    st = cycle[0]
     ses = OracleSession(sc, oracle=orc)
-    ses.apply_cache_ops(st)          # admission + writes, outside the timing
+    for s in setup + [st]:
+        ses.apply_cache_ops(s)       # admission + writes, outside the timing
     S = sc.dims.num_seqs
     t0 = time.perf_counter()
     ses.decode(st, np.arange(min(S, 4)))
@@ -250,8 +547,32 @@ def cpu_baseline(sc, seconds: float):
         if t_total > 3 * seconds:
             break
     return {"value": seqs_done / t_total, "unit": "seqs/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} x ({n} of {S} sequences: cache write of the step + float64 decode), "
-                      f"{t_total:.1f} s, {cores} OpenMP threads"}
+            "sample": f"{reps} x ({n} of {S} sequences of the first timed step: cache write of the step + "
+                      f"float64 decode), {t_total:.1f} s, {cores} OpenMP threads"}
+
+
+def also_entry(args, name, kv, rank, world, device, stream, pa, W, K):
+    """Decode time and roofline fraction of another workload, same box."""
+    import torch
+    sc = make_scenario(name, seed=1 + rank, kv=kv)
+    wl = DeviceWorkload(sc, device, None, pa, W)
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    ms_total, dec_ms, idx = wl.time_steps(K, max(3, min(args.warmup, 20)), stream, world, clocks=clocks)
+    if pa.pa_device_error(stream) != 0:
+        raise SystemExit(f"device error word set while timing {name}")
+    gbs, eff, algo, dec = wl.roofline_of(dec_ms, idx, world)
+    peak, _ = measured_hbm_peak()
+    it = wl.items[0]
+    ent = {"workload": f"{sc.name}: {sc.note}", "decode_us": dec * 1e3, "decode_gbs": gbs,
+           "frac": gbs / peak, "frac_of_8000": gbs / TARGET_GBS, "step_us": ms_total / K * 1e3,
+           "seqs_per_s": sc.dims.num_seqs * K * world / (ms_total / 1e3), "algorithmic_bytes": algo,
+           "partition_tokens": wl.P, "num_partitions": it["nparts"], "steps": K,
+           "clocks": clocks.summary()}
+    if name in ("cow", "prefix8b"):
+        ent["effective_gbs_logical"] = eff
+    del wl
+    torch.cuda.empty_cache()
+    return ent
 
 
 def run_ours(args):
@@ -269,173 +590,59 @@ def run_ours(args):
     build.build()
     from paged_kv_cache_424_b200 import binding as pa
     from paged_kv_cache_424_b200 import workload as W
-    from paged_kv_cache_424_b200.session import DeviceSession, to_device
 
-    sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv)
+    sc = make_scenario(args.workload, seed=1 + rank, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv,
+                       cycle=args.cycle)
     if args.no_prefix_order and sc.prefix_order:
         import dataclasses
         sc = dataclasses.replace(sc, prefix_order=False)
-    st = sc.steps[0]
     d = sc.dims
     fp8 = sc.kv_dtype == "fp8"
-    P = sc.partition_tokens if args.partition is None else args.partition
-    dev = DeviceSession(sc, device=str(device))
-    dev.apply_cache_ops(st)                      # prefill admission + first writes (untimed set-up)
-    inp = dev.decode_inputs(st)
-    writes = dev.write_inputs(st)
-    bm = torch.from_numpy(np.ascontiguousarray(st.block_mapping)).to(device) if st.block_mapping.size else None
-    maxlen = st.max_context_len
-    if sc.ext:
-        ws_bytes = dev.ext_workspace_bytes(inp, maxlen, P)
-        nparts = "split" if ws_bytes else 1
-    else:
-        dims = pa.dims_of(inp["q"], dev.k_cache, inp["block_tables"])
-        nparts = pa.pa_decode_num_partitions(dims, maxlen, P)
-        ws_bytes = pa.pa_decode_workspace_size(dims, maxlen, P)
-    ws = dev.workspace(ws_bytes)
-    out = torch.empty_like(inp["q"])
     stream = torch.cuda.current_stream(device)
-
-    def write(key, value, slots):
-        if fp8:
-            pa.pa_reshape_and_cache_fp8(key, value, dev.k_cache, dev.v_cache, slots, sc.k_scale, sc.v_scale,
-                                        stream=stream)
-        else:
-            pa.pa_reshape_and_cache(key, value, dev.k_cache, dev.v_cache, slots, stream=stream)
-
-    def decode(q, bt, cl, seq_order=None):
-        if sc.ext:
-            dev.decode_ext({"q": q, "block_tables": bt, "context_lens": cl, "seq_order": seq_order}, maxlen, P, out,
-                           stream=stream)
-        elif fp8:
-            pa.pa_decode_fp8(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, sc.k_scale, sc.v_scale,
-                             d.num_kv_heads, maxlen, P, ws, stream=stream)
-        else:
-            pa.pa_decode(out, q, dev.k_cache, dev.v_cache, bt, cl, sc.scale, d.num_kv_heads, maxlen, P, ws,
-                         stream=stream)
-
-    def step(e0=None, e1=None):
-        if bm is not None:
-            pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], bm, stream=stream)
-        for key, value, slots in writes:
-            write(key, value, slots)
-        if e0 is not None:
-            e0.record(stream)
-        decode(inp["q"], inp["block_tables"], inp["context_lens"], inp.get("seq_order"))
-        if e1 is not None:
-            e1.record(stream)
-
-    launches_per_step = (1 if bm is not None else 0) + len(writes) + (2 if ws_bytes else 1)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
+    wl = DeviceWorkload(sc, device, args.partition, pa, W)
     if pa.pa_device_error(stream) != 0:
-        raise SystemExit("device error word set during warm-up")
+        raise SystemExit("device error word set during set-up")
 
     K = args.steps
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(device)
-    with ClockSampler(device.index if device.index is not None else 0) as clocks:
-        start.record(stream)
-        for i in range(K):
-            step(e0[i], e1[i])
-        end.record(stream)
-        torch.cuda.synchronize(device)
-    barrier(world)
-    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
-    dec_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
-    dec_avg_ms = max_over_ranks(sum(dec_ms) / K, world, device)
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    ms_total, dec_ms, idx = wl.time_steps(K, args.warmup, stream, world, clocks=clocks)
+    if pa.pa_device_error(stream) != 0:
+        raise SystemExit("device error word set during the timed region")
+    achieved, eff_logical, algo, dec_avg_ms = wl.roofline_of(dec_ms, idx, world)
 
     # shared-prefix order: the same decode in plain batch order, for comparison
     no_order_ms = None
     if sc.prefix_order:
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for _ in range(3):
-            decode(inp["q"], inp["block_tables"], inp["context_lens"], None)
-        barrier(world)
-        torch.cuda.synchronize(device)
-        a.record(stream)
-        for _ in range(K):
-            decode(inp["q"], inp["block_tables"], inp["context_lens"], None)
-        b.record(stream)
-        torch.cuda.synchronize(device)
-        no_order_ms = max_over_ranks(a.elapsed_time(b) / K, world, device)
+        _, dec_plain, _ = wl.time_steps(K, 3, stream, world, seq_order=None)
+        no_order_ms = max_over_ranks(sum(dec_plain) / K, world, device)
 
-    # ---- end to end: host buffers in, result out, through the same calls ----
     e2e = None
     if not args.no_e2e:
-        h_q = inp["q"].cpu().pin_memory()
-        h_bt = inp["block_tables"].cpu().pin_memory()
-        h_cl = inp["context_lens"].cpu().pin_memory()
-        h_w = [(k.cpu().pin_memory(), v.cpu().pin_memory(), s.cpu().pin_memory()) for k, v, s in writes]
-        h_bm = st.block_mapping
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        d_q, d_bt, d_cl = torch.empty_like(inp["q"]), torch.empty_like(inp["block_tables"]), torch.empty_like(
-            inp["context_lens"])
-        d_w = [(torch.empty_like(k), torch.empty_like(v), torch.empty_like(s)) for k, v, s in writes]
-        h_bm_t = torch.from_numpy(np.ascontiguousarray(h_bm)).pin_memory() if bm is not None else None
-        d_bm = torch.empty_like(bm) if bm is not None else None
-        d_so = torch.empty(d.num_seqs, dtype=torch.int32, device=device) if sc.prefix_order else None
-        h_so = torch.empty(d.num_seqs, dtype=torch.int32).pin_memory() if sc.prefix_order else None
-        h2d = ((h_so.numel() * 4 if h_so is not None else 0) +
-               h_q.numel() * h_q.element_size() + h_bt.numel() * 4 + h_cl.numel() * 4 +
-               sum(k.numel() * k.element_size() * 2 + s.numel() * 8 for k, _, s in h_w) +
-               (h_bm_t.numel() * 8 if h_bm_t is not None else 0))
-        d2h = h_out.numel() * h_out.element_size()
+        e2e = wl.e2e(max(1, min(K, 500)), min(args.warmup, 10), stream, world)
+        if pa.pa_device_error(stream) != 0:
+            raise SystemExit("device error word set during the end-to-end run")
 
-        def e2e_step():
-            d_q.copy_(h_q, non_blocking=True)
-            d_bt.copy_(h_bt, non_blocking=True)
-            d_cl.copy_(h_cl, non_blocking=True)
-            for (hk, hv, hs), (dk, dv, ds) in zip(h_w, d_w):
-                dk.copy_(hk, non_blocking=True)
-                dv.copy_(hv, non_blocking=True)
-                ds.copy_(hs, non_blocking=True)
-            if d_bm is not None:
-                d_bm.copy_(h_bm_t, non_blocking=True)
-                pa.pa_copy_blocks([dev.k_cache], [dev.v_cache], d_bm, stream=stream)
-            for dk, dv, ds in d_w:
-                write(dk, dv, ds)
-            if h_so is not None:  # the host schedule of this step, then its copy
-                h_so.numpy()[:] = pa.pa_prefix_order(h_bt.numpy(), h_cl.numpy())
-                d_so.copy_(h_so, non_blocking=True)
-            decode(d_q, d_bt, d_cl, d_so)
-            h_out.copy_(out, non_blocking=True)
+    launches = sum(wl.items[j]["launches"] for j in idx)
+    it0 = wl.items[0]
+    lens = np.concatenate([wl.items[j]["step"].context_lens for j in range(len(wl.items))])
+    kv_step = sum(wl.items[j]["kv"] for j in idx) / K
+    kv_logical_step = sum(wl.items[j]["kv_logical"] for j in idx) / K
+    nparts = sorted({it["nparts"] for it in wl.items if it["nparts"] is not None})
+    C = len(wl.items)
+    kernel = ("pa_decode_ext" if sc.ext else "pa_decode_fp8" if fp8 else "pa_decode") + \
+        (" (decode kernel + log-sum-exp merge)" if any(it["ws_bytes"] for it in wl.items) else "")
+    units = float(sum(int(wl.items[j]["step"].context_lens.sum()) for j in idx)) / K
+    del wl
+    torch.cuda.empty_cache()
 
-        for _ in range(min(args.warmup, 10)):
-            e2e_step()
-        torch.cuda.synchronize(device)
-        Ke = max(1, min(K, 500))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize(device)
-        a.record(stream)
-        for _ in range(Ke):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(world)
-        e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
-        e2e = {"value": d.num_seqs * Ke * world / (e2e_ms / 1e3), "unit": "seqs/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": Ke,
-               "path": "pinned host buffers -> cudaMemcpyAsync -> pa_* C-ABI calls -> output copied back"}
+    also = {}
+    for name, kv in also_list(args):
+        key = name + ("-fp8" if kv == "fp8" else "")
+        also[key] = also_entry(args, name, kv, rank, world, device, stream, pa, W, min(max(K, 100), 500))
 
-    if pa.pa_device_error(stream) != 0:
-        raise SystemExit("device error word set during the timed region")
-
-    # Algorithmic bytes: KV of the referenced tokens; blocks shared by several
-    # sequences (copy-on-write prefixes) count once, as the pool holds them once.
-    kv_logical = W.kv_bytes(st, d, elem_bytes=sc.kv_elem_bytes, q_len=sc.q_len, window=sc.window)
-    kv = (W.kv_bytes(st, d, unique=True, elem_bytes=sc.kv_elem_bytes) if args.workload in ("cow", "prefix8b")
-          else kv_logical)
-    algo = kv + W.qo_bytes(d, sc.q_len)
+    part_tokens = sc.partition_tokens if args.partition is None else args.partition
     peak, peak_kind = measured_hbm_peak()
-    achieved = algo / (dec_avg_ms / 1e3) / 1e9
-    traffic = ncu_traffic(args.workload + ("-fp8" if fp8 else ""), units=float(st.context_lens.sum()))
+    traffic = ncu_traffic(args.workload + ("-fp8" if fp8 else ""), units=units)
     result = {
         "metric": METRIC,
         "value": d.num_seqs * K * world / (ms_total / 1e3),
@@ -450,26 +657,27 @@ def run_ours(args):
         "dtype": f"{d.dtype} q/out, e4m3 KV cache" if fp8 else d.dtype,
         "data": "synthetic (seeded U[-1,1] fp16/bf16 values, NaN in every unused slot; no dataset)",
         "config": {"workload": f"{sc.name}: {sc.note}", "global_batch": d.num_seqs * world,
-                   "seq_len": "per-sequence, " + f"mean {float(st.context_lens.mean()):.0f}, "
-                              f"max {int(st.context_lens.max())}",
-                   "partition_tokens": P, "num_partitions": nparts,
+                   "seq_len": f"per-sequence, mean {float(lens.mean()):.0f}, max {int(lens.max())} over the cycle",
+                   "timed_cycle": (f"{C} churned steps (after 2 set-up steps), walked in turn: each timed step "
+                                   f"decodes a different batch mix" if C > 1 else "one step, repeated"),
+                   "partition_tokens": part_tokens or "auto",
+                   "num_partitions": nparts if nparts else "split" if "merge" in kernel else 1,
                    **({"q_len": sc.q_len, "window": sc.window} if sc.ext else {}),
                    **({"seq_order": "pa_prefix_order", "decode_ms_batch_order": no_order_ms,
                        "decode_ms_prefix_order": dec_avg_ms,
                        "prefix_order_speedup": no_order_ms / dec_avg_ms} if no_order_ms else {}),
                    "parallelism": f"{world} independent batches (one per GPU, no data-path collective)",
-                   "l2": f"inputs larger than L2: {kv / 1e9:.2f} GB of KV read per step vs 126 MB L2",
-                   "kv_bytes_per_step": kv, "kv_bytes_logical_per_step": kv_logical,
-                   "algorithmic_bytes_per_step": algo},
+                   "l2": f"inputs larger than L2: {kv_step / 1e9:.2f} GB of KV read per step vs 126 MB L2",
+                   "kv_bytes_per_step": kv_step, "kv_bytes_logical_per_step": kv_logical_step,
+                   "algorithmic_bytes_per_step": algo,
+                   **({"also": also} if also else {})},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": ("pa_decode_ext" if sc.ext else "pa_decode_fp8" if fp8 else "pa_decode") +
-                               (" (decode kernel + log-sum-exp merge)" if ws_bytes else ""),
-                     "kernel_ms": dec_avg_ms, "frac_of_8000": achieved / 8000.0,
-                     "effective_gbs_logical": (kv_logical + W.qo_bytes(d, sc.q_len)) / (dec_avg_ms / 1e3) / 1e9},
+                     "kernel": kernel, "kernel_ms": dec_avg_ms, "frac_of_8000": achieved / TARGET_GBS,
+                     "effective_gbs_logical": eff_logical},
         "clocks": clocks.summary(),
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": launches,
     }
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(sc, args.cpu_seconds)
@@ -491,18 +699,21 @@ def run_reference(args):
     from oracle.harness import OracleSession
     orc = oracle.load()
     cores = orc.max_threads()
-    sc = make_scenario(args.workload, seed=1, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv)
-    st = sc.steps[0]
+    sc = make_scenario(args.workload, seed=1, num_seqs=args.num_seqs, num_blocks=args.num_blocks, kv=args.kv,
+                       cycle=args.cycle)
+    setup, cycle = scenario_cycle(sc)
     S = sc.dims.num_seqs
     ses = OracleSession(sc, oracle=orc)
-    ses.apply_cache_ops(st)
+    for st in setup + cycle:
+        ses.apply_cache_ops(st)
     t0 = time.perf_counter()
-    ses.decode(st, np.arange(min(S, 2)))
+    ses.decode(cycle[0], np.arange(min(S, 2)))
     t_seq = (time.perf_counter() - t0) / min(S, 2)
     budget = 120.0 / max(1, args.steps + args.warmup)          # seconds per step
     n = int(max(1, min(S, budget / max(t_seq, 1e-9))))
 
     def one(i):
+        st = cycle[i % len(cycle)]
         sel = (np.arange(n) + i * n) % S
         for w in st.writes:
             ses.write(w.key, w.value, w.slot_mapping)
@@ -512,10 +723,11 @@ def run_reference(args):
         one(i)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        one(i)
+        one(args.warmup + i)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
-    sample = f"each step: {n} of {S} sequences (cache write + float64 decode), {cores} OpenMP threads"
+    sample = (f"each step: {n} of {S} sequences of the step's batch (cache write + float64 decode), walking the "
+              f"{len(cycle)}-step cycle, {cores} OpenMP threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
