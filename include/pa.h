@@ -173,6 +173,9 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  *   partial result it later reads), but calls whose kernels overlap on the
  *   GPU (different streams, or several host threads) race on it: order them
  *   on one stream or use pa_decode with separate workspaces.
+ * - If a pipeline wait gives up (PA_DEVERR_TIMEOUT in pa_device_error), the
+ *   output of that call is undefined: the merge may have read partial
+ *   results an earlier call left in the shared array.
  * Results are those of pa_decode with the same arguments.
  */
 pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -186,17 +189,14 @@ pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const
  * weights ("vLLM PagedAttention 大模型推理架构深度实战" section 5.2) and
  * KV-cache compression as a goal (section 九 item 3).  Same definition as
  * pa_decode with K_s[j] = decode(k code) * k_scale and V_s[j] = decode(v code)
- * * v_scale; q / out in dims->dtype.  Groups of 4, 8 or 16 query heads at
- * head_dim 128 run on the tensor-core kernel; other shapes on the CUDA-core
- * kernel.  With 4 or 8 rows per KV head the tensor cores multiply the E4M3
- * codes as stored: q is split into three E4M3 parts under a power-of-two
- * factor per row (q recovered to within 2^-15 of the row's largest |q|, any
- * finite q) and the softmax weights w into four (|error| <= 2^-12 w +
- * 2^-22).  With 16 rows (group 16, or several query tokens through
- * pa_decode_ext) the codes are widened in shared memory to f16 and q is
- * converted to f16 for the MMA: a bf16 q must then lie within f16's range,
- * |q| <= 65504, and loses precision below 2^-14.
- * Workspace as from pa_decode_workspace_size with the same dims.
+ * * v_scale; q / out in dims->dtype.  With 4, 8 or 16 query rows per KV
+ * head (the group, or group x query tokens through pa_decode_ext) at
+ * head_dim 128 the tensor cores multiply the E4M3 codes as stored: q is
+ * split into three E4M3 parts under a power-of-two factor per row (q
+ * recovered to within 2^-15 of the row's largest |q|, for any finite q,
+ * fp16 or bf16) and the softmax weights w into four (|error| <= 2^-12 w +
+ * 2^-22).  Other shapes run on the CUDA-core kernel, which widens each code
+ * exactly.  Workspace as from pa_decode_workspace_size with the same dims.
  */
 pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
                         const int32_t *block_tables, const int32_t *context_lens, float scale,

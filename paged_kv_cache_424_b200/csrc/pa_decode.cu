@@ -148,9 +148,12 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
     state.init();
     float *pw = p_s + warp * G * kBlock;
     bool ok = true;
-    for (int j = 0; j < nw; ++j) {
+    int j = 0;
+    for (; j < nw; ++j) {
         const int st = j % NSTAGE;
-        if (!mbar_wait(&wbar[st], (j / NSTAGE) & 1)) {
+        // warp-uniform: every lane takes the same branch even if the copy lands
+        // just as some lanes give up
+        if (!__all_sync(0xffffffffu, mbar_wait(&wbar[st], (j / NSTAGE) & 1))) {
             ok = false;
             break;
         }
@@ -163,9 +166,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
         }
     }
     if (!ok) {
-        // A copy never completed (the error word is set).  Give it one more
-        // bounded chance to land before the CTA exits; write nothing.
-        if (lane == 0) mbar_wait(&wbar[0], 0, 200000000ll);
+        // A copy never completed (the error word is set).  Every copy issued
+        // into this warp's ring and not yet consumed (blocks j .. j + NSTAGE - 1)
+        // gets one more bounded chance to land before the CTA exits, so none
+        // can still be writing into shared memory afterwards; write nothing.
+        if (lane == 0)
+            for (int jj = j; jj < j + NSTAGE && jj < nw; ++jj)
+                mbar_wait(&wbar[jj % NSTAGE], (jj / NSTAGE) & 1, 200000000ll);
         atomicOr(&fail_s, 1);
     }
 
@@ -203,12 +210,89 @@ __global__ void __launch_bounds__(kWarps * 32) decode_part_kernel(const DecodePa
 
 // out[row, :] = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p,
 // over the partitions sequence s actually uses (all -inf: a masked row with
-// no position, zero).  A CTA of D threads takes `rows_per_cta` consecutive
-// rows (query token x head) of sequence s, so a batch with many rows pays
-// the per-sequence check and the launch once per group of rows.
+// no position, zero).  A CTA of 4 warps takes `rows_per_cta` consecutive rows
+// (query token x head) of sequence s.  A lane holds D / 32 consecutive dims,
+// so a warp reads one partition's row of o with one coalesced load, and up
+// to kInFlight partitions' loads are issued before the first is used.  With
+// few partitions (<= kWarpRowParts) each warp merges whole rows on its own;
+// with more, the 4 warps share a row (warp w takes partitions w, w + 4, ...)
+// and add their sums in shared memory.
+constexpr int kMergeWarps = 4;
+constexpr int kInFlight = 8;
+constexpr int kWarpRowParts = 8;
+
+template <int D>
+struct MergeAcc {
+    static constexpr int kV = D / 32;  // dims per lane
+    float o[kV];
+    float w;  // sum of the weights seen
+};
+
+// Weighted sum of partitions first, first + stride, ... < n of one row into
+// `a` (lane's dims); M is the row's max lse (finite).
+template <int D>
+__device__ __forceinline__ void merge_accumulate(MergeAcc<D> &a, const float *lse, const float *o_row, int first,
+                                                 int stride, int n, float M, int lane) {
+    constexpr int kV = MergeAcc<D>::kV;
+    for (int i0 = first; i0 < n; i0 += stride * kInFlight) {
+        float w[kInFlight];
+        float v[kInFlight][kV];
+#pragma unroll
+        for (int k = 0; k < kInFlight; ++k) {
+            const int i = i0 + k * stride;
+            w[k] = 0.f;
+#pragma unroll
+            for (int e = 0; e < kV; ++e) v[k][e] = 0.f;
+            if (i < n) {
+                w[k] = exp2f(lse[i] - M);  // lse = -inf (no position in that partition) gives 0
+                const float *src = o_row + (int64_t)i * D + lane * kV;
+                if constexpr (kV == 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(src);
+                    v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+                } else {
+                    const float2 x = *reinterpret_cast<const float2 *>(src);
+                    v[k][0] = x.x; v[k][1] = x.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kInFlight; ++k) {
+            a.w += w[k];
+#pragma unroll
+            for (int e = 0; e < kV; ++e) a.o[e] = fmaf(w[k], v[k][e], a.o[e]);
+        }
+    }
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p, const int rows_per_cta) {
-    const int s = blockIdx.y, d = threadIdx.x;
+__device__ __forceinline__ void merge_store(T *out, int lane, const float *o, float wsum) {
+    constexpr int kV = D / 32;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    if constexpr (kV == 4) {
+        const typename Elem<T>::T2 a = {Elem<T>::from_float(o[0] * inv), Elem<T>::from_float(o[1] * inv)};
+        const typename Elem<T>::T2 b = {Elem<T>::from_float(o[2] * inv), Elem<T>::from_float(o[3] * inv)};
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&a);
+        u.y = *reinterpret_cast<const uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(out + lane * kV) = u;
+    } else {
+        const typename Elem<T>::T2 a = {Elem<T>::from_float(o[0] * inv), Elem<T>::from_float(o[1] * inv)};
+        *reinterpret_cast<typename Elem<T>::T2 *>(out + lane * kV) = a;
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_part_kernel(const DecodeParams p, const int rows_per_cta) {
+    constexpr int kV = MergeAcc<D>::kV;
+    __shared__ float red_o[kMergeWarps][D];
+    __shared__ float red_w[kMergeWarps];
+    const int s = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
     pdl_wait();
     const SeqSplit sp = seq_split(p, s, false);
@@ -217,22 +301,50 @@ __global__ void __launch_bounds__(D) merge_part_kernel(const DecodeParams p, con
     const int rows = p.q_len * p.num_heads;
     const int r0 = blockIdx.x * rows_per_cta;
     const int r1 = min(r0 + rows_per_cta, rows);
+    T *out = reinterpret_cast<T *>(p.out);
+    auto row_max = [&](const float *lse) {
+        float M = -INFINITY;
+        for (int i = lane; i < nparts; i += 32) M = fmaxf(M, lse[i]);
+        return warp_max(M);
+    };
+    if (nparts <= kWarpRowParts) {
+        // a warp per row
+        for (int r = r0 + warp; r < r1; r += kMergeWarps) {
+            const int64_t qr = (int64_t)s * rows + r;
+            const float *lse = p.ws_lse + qr * p.max_parts;
+            const float M = row_max(lse);
+            MergeAcc<D> a{};
+            if (M != -INFINITY) merge_accumulate<D>(a, lse, p.ws_o + qr * p.max_parts * D, 0, 1, nparts, M, lane);
+            merge_store<T, D>(out + qr * D, lane, a.o, a.w);
+        }
+        return;
+    }
+    // the CTA's 4 warps per row
     for (int r = r0; r < r1; ++r) {
         const int64_t qr = (int64_t)s * rows + r;
-        const int64_t row = qr * p.max_parts;
-        const float *lse = p.ws_lse + row;
-        float M = -INFINITY;
-        for (int i = 0; i < nparts; ++i) M = fmaxf(M, lse[i]);
-        float wsum = 0.f, o = 0.f;
-        if (M != -INFINITY) {
-            for (int i = 0; i < nparts; ++i) {
-                const float w = exp2f(lse[i] - M);
-                wsum += w;
-                o = fmaf(w, p.ws_o[(row + i) * D + d], o);
+        const float *lse = p.ws_lse + qr * p.max_parts;
+        const float M = row_max(lse);
+        MergeAcc<D> a{};
+        if (M != -INFINITY)
+            merge_accumulate<D>(a, lse, p.ws_o + qr * p.max_parts * D, warp, kMergeWarps, nparts, M, lane);
+#pragma unroll
+        for (int e = 0; e < kV; ++e) red_o[warp][lane * kV + e] = a.o[e];
+        if (lane == 0) red_w[warp] = a.w;
+        __syncthreads();
+        if (warp == 0) {
+            float o[kV];
+#pragma unroll
+            for (int e = 0; e < kV; ++e) {
+                o[e] = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMergeWarps; ++w) o[e] += red_o[w][lane * kV + e];
             }
-            o /= wsum;
+            float wsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; ++w) wsum += red_w[w];
+            merge_store<T, D>(out + qr * D, lane, o, wsum);
         }
-        reinterpret_cast<T *>(p.out)[qr * D + d] = Elem<T>::from_float(o);
+        __syncthreads();
     }
 }
 
@@ -242,8 +354,8 @@ cudaError_t launch_part_m(const DecodeParams &p, cudaStream_t stream) {
     constexpr int kStages = part_stages(G, kEsz);
     auto kern = decode_part_kernel<T, KT, D, G, kStages, kMasked>;
     const int smem = PartLayout(D, G, kStages, kEsz).bytes(p.part_blocks);
-    static int configured[kMaxDevices] = {};
-    cudaError_t e = ensure_smem(kern, smem, configured);
+    static FuncAttrCache attrs;
+    cudaError_t e = ensure_smem(kern, smem, attrs);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3(p.max_parts, p.num_kv_heads, p.num_seqs), dim3(kWarps * 32), smem, stream, p);
     if (e != cudaSuccess || p.max_parts == 1) return e;
@@ -276,18 +388,26 @@ cudaError_t launch_part_k(const DecodeParams &p, int head_dim, int group, cudaSt
 }  // namespace
 
 cudaError_t launch_merge_partitions(const DecodeParams &p, int dtype, int head_dim, cudaStream_t stream) {
-    // Rows per CTA: 1 while the grid stays under ~4 waves of small CTAs,
-    // up to 8 for batches with many rows (multi-token queries).
+    // Rows per CTA: with few partitions a warp merges a row on its own, so a
+    // CTA takes 4 rows (up to 16 for batches with many rows, e.g. several
+    // query tokens); with many partitions the 4 warps share a row and a CTA
+    // takes 1 row (up to 8 for very large batches).
     const int64_t rows = (int64_t)p.num_heads * p.q_len;
     const int64_t total = rows * p.num_seqs;
     int rpc = 1;
-    while (rpc < 8 && total / (rpc * 2) >= 8192) rpc *= 2;
+    if (p.max_parts <= kWarpRowParts) {
+        rpc = kMergeWarps;
+        while (rpc < 16 && total / (rpc * 2) >= 4096) rpc *= 2;
+    } else {
+        while (rpc < 8 && total / (rpc * 2) >= 8192) rpc *= 2;
+    }
     const dim3 grid((unsigned)((rows + rpc - 1) / rpc), p.num_seqs);
+    const dim3 block(kMergeWarps * 32);
     if (dtype == PA_F16)
-        return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, dim3(64), 0, stream, p, rpc)
-                              : launch_pdl(merge_part_kernel<__half, 128>, grid, dim3(128), 0, stream, p, rpc);
-    return head_dim == 64 ? launch_pdl(merge_part_kernel<__nv_bfloat16, 64>, grid, dim3(64), 0, stream, p, rpc)
-                          : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, stream, p, rpc);
+        return head_dim == 64 ? launch_pdl(merge_part_kernel<__half, 64>, grid, block, 0, stream, p, rpc)
+                              : launch_pdl(merge_part_kernel<__half, 128>, grid, block, 0, stream, p, rpc);
+    return head_dim == 64 ? launch_pdl(merge_part_kernel<__nv_bfloat16, 64>, grid, block, 0, stream, p, rpc)
+                          : launch_pdl(merge_part_kernel<__nv_bfloat16, 128>, grid, block, 0, stream, p, rpc);
 }
 
 cudaError_t launch_decode_partitioned(const DecodeParams &p, int dtype, int head_dim, int rows, bool fp8_cache,

@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/pa.h"
 
 namespace pa {
@@ -38,18 +41,38 @@ struct DecodeParams {
 // sliding window); the kernels take this as a template flag.
 inline bool decode_masked(const DecodeParams &p) { return p.q_len != 1 || p.window != 0; }
 
+// Per-device record of the function attributes a kernel has been given
+// (one per kernel instantiation).  Launches may come from several host
+// threads: the fast path is one atomic load, and the attribute calls run
+// under a lock so the recorded value never exceeds what was really set.
+struct FuncAttrCache {
+    std::atomic<int> smem[kMaxDevices] = {};      // dynamic shared-memory limit set
+    std::atomic<int> carveout[kMaxDevices] = {};  // 1 once the carveout preference is set
+    std::mutex mu;
+};
+
 // Raise a kernel's dynamic shared-memory limit on the current device when a
-// launch needs more than was set before (the attribute is per device).
+// launch needs more than was set before (the attribute is per device), and
+// optionally ask for the largest shared-memory carveout once.
 template <typename K>
-inline cudaError_t ensure_smem(K kern, int bytes, int *configured_per_device) {
+inline cudaError_t ensure_smem(K kern, int bytes, FuncAttrCache &cache, bool max_carveout = false) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (bytes > 48 * 1024 && bytes > configured_per_device[dev]) {
+    const bool need_smem = bytes > 48 * 1024 && bytes > cache.smem[dev].load(std::memory_order_acquire);
+    const bool need_carveout = max_carveout && !cache.carveout[dev].load(std::memory_order_acquire);
+    if (!need_smem && !need_carveout) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(cache.mu);
+    if (max_carveout && !cache.carveout[dev].load(std::memory_order_relaxed)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        cache.carveout[dev].store(1, std::memory_order_release);
+    }
+    if (bytes > 48 * 1024 && bytes > cache.smem[dev].load(std::memory_order_relaxed)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
-        configured_per_device[dev] = bytes;
+        cache.smem[dev].store(bytes, std::memory_order_release);
     }
     return cudaSuccess;
 }

@@ -30,12 +30,12 @@
 //           tile, and accumulates O chunk by chunk in registers.
 // Shared memory: K tile 32 KiB + V tile 32 KiB + Q 4 KiB + P 4 KiB (+ <1 KiB)
 // = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
-// FP8 E4M3 caches, groups of 4 or 8: the K and V tiles hold the chunk's
-// codes as loaded (16 KiB each, 128-byte swizzle) and both products run
-// E4M3 x E4M3: S = K . Q^T against Q split into three E4M3 parts (3G
-// columns), O^T = V^T . P^T against P split into four (4G columns); S and
-// O take 4G columns each, 64 or 128 TMEM columns in all.  FP8 with 16
-// columns widens K and V to f16 in place.
+// FP8 E4M3 caches: a chunk's codes take 16 KiB (128-byte swizzle), so each
+// 32 KiB tile area holds two stages and the loads of chunk c + 1 overlap the
+// products of chunk c.  Both products run E4M3 x E4M3 on the codes as
+// loaded: S = K . Q^T against Q split into three E4M3 parts (3G columns,
+// rounded up to 16), O^T = V^T . P^T against P split into four (4G
+// columns); 64, 128 or 256 TMEM columns for G = 4, 8, 16.
 // Results go to `out` (one partition) or to the split workspace for the
 // log-sum-exp merge, exactly like the CUDA-core kernel.
 #include <cfloat>
@@ -53,35 +53,53 @@ namespace pa {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kN = 16;              // MMA N: query heads padded to 16
+constexpr int kN = 16;              // MMA N of a 16-bit cache: query rows padded to 16
 constexpr int kChunk = 128;         // tokens per chunk (MMA M)
 constexpr int kChunkBlocks = kChunk / kBlock;
-constexpr int kRegion = kChunk * 128;   // one 64-dim half of a K or V tile (bytes)
+constexpr int kRegion = kChunk * 128;   // one 64-dim half of a 16-bit K or V tile, or one chunk of E4M3 codes (bytes)
 
-// Shared-memory layout (bytes from the 1024-aligned base).
-constexpr int kKOff = 0;
-constexpr int kVOff = kKOff + 2 * kRegion;      // 32768
-constexpr int kQOff = kVOff + 2 * kRegion;      // 65536
-constexpr int kPOff = kQOff + 2 * kN * 128;     // 69632
-constexpr int kRedOff = kPOff + 2 * kN * 128;   // 73728: [2][4][16] floats
-constexpr int kBarOff = kRedOff + 2 * 4 * kN * 4;
-constexpr int kNumBars = 12;
-constexpr int kMiscOff = kBarOff + kNumBars * 8;  // TMEM base, fail flag, 4 lazy-max flags
-constexpr int kQScaleOff = kMiscOff + 32;          // FP8 with E4M3 products: [8] per-row logit factors
-constexpr int kSmemTc = kQScaleOff + 32;
-
-// FP8 caches with groups of 4 or 8 run both products on the E4M3 codes as
-// loaded: Q is split into three E4M3 parts and P into four, stacked as 3G
-// and 4G columns, so S and O have NS = 4G = 16 or 32 columns.  TMEM: S
-// buffers at 0 and NS, O buffers at 2 NS and 3 NS; 64 columns (128 with
-// NS = 32).
+// FP8 caches run both products on the E4M3 codes as loaded: Q is split into
+// three E4M3 parts and P into four, stacked as 3G and 4G columns, so S has
+// NSq = 3G columns rounded up to the MMA's N granule of 16 and O has NSo =
+// 4G.  TMEM: four buffers (S twice, then O twice), each starting at a
+// multiple of its power-of-two stride: 16 columns each for G = 4 (64 in
+// all), 32 for G = 8 (128), 64 for G = 16 (256).
 constexpr int kQParts = 3, kPParts = 4;
-__host__ __device__ constexpr int tc_cols(int G, bool e4m3) { return e4m3 && G > 4 ? 32 : kN; }
-__host__ __device__ constexpr uint32_t tc_tmem_cols(int ns) { return 4 * ns <= 64 ? 64u : 128u; }
-template <int NS>
-__device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * NS); }
-template <int NS>
-__device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)(2 * NS + b * NS); }
+__host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
+__host__ __device__ constexpr int pow2_at_least(int x) { return x <= 16 ? 16 : x <= 32 ? 32 : x <= 64 ? 64 : 128; }
+__host__ __device__ constexpr int tc_cols_s(int G, bool e4m3) { return e4m3 ? round16(kQParts * G) : kN; }
+__host__ __device__ constexpr int tc_cols_o(int G, bool e4m3) { return e4m3 ? kPParts * G : kN; }
+__host__ __device__ constexpr int tc_buf_stride(int nsq, int nso) { return pow2_at_least(nsq > nso ? nsq : nso); }
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int nsq, int nso) {
+    return 4 * tc_buf_stride(nsq, nso) < 32 ? 32u : (uint32_t)(4 * tc_buf_stride(nsq, nso));
+}
+template <int NSq, int NSo>
+__device__ __forceinline__ uint32_t s_col(int b) { return (uint32_t)(b * tc_buf_stride(NSq, NSo)); }
+template <int NSq, int NSo>
+__device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)((2 + b) * tc_buf_stride(NSq, NSo)); }
+static_assert(tc_tmem_cols(16, 16) == 64 && tc_tmem_cols(32, 32) == 128 && tc_tmem_cols(48, 64) == 256,
+              "TMEM columns per CTA");
+
+// K / V stages: a 16-bit chunk fills its 32 KiB tile area (two 64-dim
+// regions), one stage; E4M3 codes take 16 KiB, so each area holds two
+// stages and the loads of chunk c + 1 overlap the products of chunk c.
+__host__ __device__ constexpr int tc_stages(bool e4m3) { return e4m3 ? 2 : 1; }
+__host__ __device__ constexpr int tc_stage_bytes(bool e4m3) { return e4m3 ? kRegion : 2 * kRegion; }
+
+// Shared-memory layout (bytes from the 1024-aligned base): K tile area,
+// V tile area, Q tile (16-bit: two 64-dim regions of 16 rows; E4M3: NSq
+// rows of 128 codes), P tile (16-bit: two 64-token regions of 16 rows;
+// E4M3: NSo rows of 128 codes), the cross-warp reduction [2][4][16] floats,
+// the mbarriers, TMEM base / fail flag / 4 lazy-max flags, and the per-row
+// logit factors of the E4M3 path.
+constexpr int kNumBars = 16;
+struct TcLayout {
+    int k_off, v_off, q_off, p_off, red_off, bar_off, misc_off, qscale_off, bytes;
+    __host__ __device__ constexpr TcLayout(int G, bool e4m3)
+        : k_off(0), v_off(2 * kRegion), q_off(4 * kRegion), p_off(q_off + (e4m3 ? tc_cols_s(G, true) * 128 : 2 * kN * 128)),
+          red_off(p_off + (e4m3 ? tc_cols_o(G, true) * 128 : 2 * kN * 128)), bar_off(red_off + 2 * 4 * kN * 4),
+          misc_off(bar_off + kNumBars * 8), qscale_off(misc_off + 32), bytes(qscale_off + kN * 4) {}
+};
 
 __device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
 
@@ -103,43 +121,66 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// One producer warp streams one of the two tiles (K or V) chunk by chunk:
-// wait until the MMA that read the tile's previous chunk has completed
-// (`empty`), then load the chunk's 8 blocks (zeros past the partition).
-// The table slice is held in registers, 32 entries per window, the next
-// window prefetched one window ahead.  kCodes: the tile holds E4M3 codes,
-// one 128-byte row per token (one box per block) instead of two 64-dim
-// regions of 16-bit elements.
-template <bool kCodes = false>
+// One producer warp streams one of the two tiles (K or V) chunk by chunk
+// through kStages stages: wait until the MMA that read the stage's previous
+// chunk has completed (`empty[stage]`), then load the chunk's 8 blocks
+// (zeros past the partition) completing on `full[stage]`.  The table slice
+// is held in registers, 32 entries per window, the next window prefetched
+// one window ahead.  kCodes: the tile holds E4M3 codes, one 128-byte row per
+// token (one box per block) instead of two 64-dim regions of 16-bit elements.
+// The first two 32-entry windows of a producer's table slice, loaded before
+// the context length is known (entries past the slice are read, when they
+// lie inside the table row, and ignored).
+struct TablePrefetch {
+    bool valid;
+    int32_t w0, w1;
+};
+
+template <bool kCodes, int kStages>
 __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
                                              uint64_t *full, uint64_t *empty, int *fail, int s, int kvh, int b0,
-                                             int nb, int nch, int oob_row, int lane) {
+                                             int nb, int nch, int oob_row, int lane, const TablePrefetch &pre) {
+    constexpr int kStageBytes = tc_stage_bytes(kCodes);
     const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
+    auto slot_of = [&](int bi, int32_t entry) -> int {
+        return bi < nb ? (int)((checked_block(p, entry) * p.num_kv_heads + kvh) * kBlock) : oob_row;
+    };
     auto window = [&](int w) -> int {
         const int bi = w * 32 + lane;
-        return bi < nb ? (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock) : oob_row;
+        return slot_of(bi, bi < nb ? row[bi] : 0);
     };
     if (lane == 0) prefetch_tmap(tmap);
-    int cur = window(0);
-    int next = nb > 32 ? window(1) : oob_row;
+    int cur = pre.valid ? slot_of(lane, pre.w0) : window(0);
+    int next = nb > 32 ? (pre.valid ? slot_of(32 + lane, pre.w1) : window(1)) : oob_row;
+    int issued = 0;
     for (int c = 0; c < nch; ++c) {
         if (c > 0 && (c & 3) == 0) {
             cur = next;
             next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1) : oob_row;
         }
         const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
+        const int st = c % kStages;
         bool ok = true;
         if (lane == 0) {
-            ok = c == 0 || wait_ok(empty, (c - 1) & 1, fail);
-            if (ok) mbar_arrive_expect_tx(full, kCodes ? kRegion : 2 * kRegion);
+            ok = c < kStages || wait_ok(&empty[st], (c / kStages - 1) & 1, fail);
+            if (ok) mbar_arrive_expect_tx(&full[st], kCodes ? kRegion : 2 * kRegion);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        unsigned char *dst = tile + st * kStageBytes;
         if (lane < kChunkBlocks) {
-            tc::tma_load_2d(tile + lane * 2048, tmap, 0, y, full);
-            if constexpr (!kCodes) tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 64, y, full);
+            tc::tma_load_2d(dst + lane * 2048, tmap, 0, y, &full[st]);
+            if constexpr (!kCodes) tc::tma_load_2d(dst + kRegion + lane * 2048, tmap, 64, y, &full[st]);
         }
+        issued = c + 1;
     }
+    // After a failure the last chunks issued may still be landing (their
+    // consumer gave up): give each a bounded chance before the CTA exits.
+    // At most kStages chunks are outstanding: chunk c is issued only after
+    // chunk c - kStages was consumed.
+    if (lane == 0 && is_failed(fail))
+        for (int c = issued - kStages > 0 ? issued - kStages : 0; c < issued; ++c)
+            mbar_wait(&full[c % kStages], (c / kStages) & 1, 200000000ll);
 }
 
 // Softmax warps: one per TMEM lane quadrant, each thread holding the state
@@ -148,81 +189,6 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
 // producer, the MMA issuer and the V producer.
 __host__ __device__ constexpr int tc_soft_warps(int G) { return G > 8 ? 8 : 4; }
 __host__ __device__ constexpr int tc_threads(int G) { return (tc_soft_warps(G) + 3) * 32; }
-// FP8 E4M3 caches: the producer loads a chunk's codes (128 tokens x 128
-// bytes) by TMA into the second 64-dim region of the 16-bit tile and
-// converts them there into the tile's f16 layout (codes widen exactly to
-// f16).  A step reads 16 rows of codes (four 512-byte runs, four
-// independent 16-byte loads per lane) before it writes those 16 rows of
-// f16: a row's f16 lands in both regions at the same row, over its own codes
-// only, so no code is overwritten before it is read.
-__device__ __forceinline__ void convert_fp8_chunk(unsigned char *tile, int lane) {
-    const unsigned char *codes = tile + kRegion;
-    const int c16 = lane & 7;  // codes [16 c16, 16 c16 + 16) of the row = dims
-    unsigned char *dst = tile + (c16 >> 2) * kRegion;
-    const int col = (c16 & 3) * 16;  // first element of those dims within their region
-    constexpr int kRowsPerStep = 16;  // 4 independent 16-byte loads per lane in flight
-#pragma unroll 1
-    for (int step = 0; step < kChunk / kRowsPerStep; ++step) {
-        uint4 raw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            raw[k] = *reinterpret_cast<const uint4 *>(codes + (step * kRowsPerStep + k * 4 + (lane >> 3)) * 128 +
-                                                      c16 * 16);
-        __syncwarp();  // all 16 rows read before any of them is overwritten
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = step * kRowsPerStep + k * 4 + (lane >> 3);
-            const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-            uint32_t h[8];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint16_t lo, hi;
-                split_b32(w[j], lo, hi);
-                h[2 * j] = e4m3x2_to_half2_bits(lo);
-                h[2 * j + 1] = e4m3x2_to_half2_bits(hi);
-            }
-            *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4 *>(dst + tc::sw128_offset(r, col + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
-        }
-        __syncwarp();
-    }
-}
-
-// The producer of an FP8 tile: per chunk, wait until the MMA that read the
-// tile's previous chunk has completed, load the chunk's codes into the
-// tile's second region (`stage` completes the copies), convert, and arrive
-// on `full` (32 arrivals: one per lane).
-__device__ __forceinline__ void produce_tile_fp8(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
-                                                 uint64_t *stage, uint64_t *full, uint64_t *empty, int *fail, int s,
-                                                 int kvh, int b0, int nb, int nch, int oob_row, int lane) {
-    const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
-    auto window = [&](int w) -> int {
-        const int bi = w * 32 + lane;
-        return bi < nb ? (int)((checked_block(p, row[bi]) * p.num_kv_heads + kvh) * kBlock) : oob_row;
-    };
-    if (lane == 0) prefetch_tmap(tmap);
-    int cur = window(0);
-    int next = nb > 32 ? window(1) : oob_row;
-    for (int c = 0; c < nch; ++c) {
-        if (c > 0 && (c & 3) == 0) {
-            cur = next;
-            next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1) : oob_row;
-        }
-        const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
-        bool ok = true;
-        if (lane == 0) {
-            ok = c == 0 || wait_ok(empty, (c - 1) & 1, fail);
-            if (ok) mbar_arrive_expect_tx(stage, kChunk * 128);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        if (lane < kChunkBlocks) tc::tma_load_2d(tile + kRegion + lane * 2048, tmap, 0, y, stage);
-        if (!__all_sync(0xffffffffu, wait_ok(stage, c & 1, fail))) break;
-        convert_fp8_chunk(tile, lane);
-        fence_proxy_async_smem();  // the f16 tile is read by the MMA (async proxy)
-        mbar_arrive(full);
-    }
-}
 
 // CTAs per SM: 3 (registers and shared memory both allow it) except with 16
 // columns, whose 11 warps fit twice.
@@ -231,44 +197,43 @@ __host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; 
 // G: columns of S (query rows per KV head: the group, or group x query
 // tokens with kMasked, padded to a power of two).
 // kFp8: the caches hold E4M3 codes; k_scale sits in scale_log2 and v_scale
-// multiplies the output.  With G = 4 or 8 both products run E4M3 x E4M3 on
-// the codes as loaded: Q is split into three E4M3 parts with one
-// power-of-two factor per query row (4 + 4 + 4 significant bits recover a
-// 16-bit q to within 2^-15 of the row's largest |q|), P into four parts
-// (|w - sum| <= 2^-12 w + 2^-22); the f32 products of the parts are
-// recombined when S and O are read from TMEM.  With 16 columns K and V are
-// widened to f16 in place and both products run f16 x f16 (q converted to
-// f16 on load).
+// multiplies the output.  Both products run E4M3 x E4M3 on the codes as
+// loaded, two stages per tile: Q is split into three E4M3 parts with one
+// power-of-two factor per query row (4 + 4 + 4 significant bits recover any
+// finite 16-bit q to within 2^-15 of the row's largest |q|), P into four
+// parts (|w - sum| <= 2^-12 w + 2^-22); the f32 products of the parts are
+// recombined when S and O are read from TMEM.
 template <typename T, int G, bool kMasked, bool kFp8>
 __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
     static_assert(!kFp8 || kMasked, "FP8 launches take the masked variant (it applies v_scale)");
     using E = Elem<T>;
-    using MT = typename std::conditional<kFp8, __half, T>::type;  // type of the MMA operands
-    using EM = Elem<MT>;
-    constexpr bool kBf16 = std::is_same<MT, __nv_bfloat16>::value;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int kSW = tc_soft_warps(G);       // softmax warps
     constexpr int kST = kSW * 32;                // softmax threads
     constexpr int kGT = G > 8 ? 8 : G;           // columns per softmax thread
     constexpr int kWarpK = kSW, kWarpMma = kSW + 1, kWarpV = kSW + 2;
-    constexpr bool kE4m3 = kFp8 && G <= 8;       // both products on the E4M3 codes
-    constexpr int kNS = tc_cols(G, kE4m3);       // columns of S and O
-    constexpr uint32_t kTmemCols = tc_tmem_cols(kNS);
+    constexpr bool kE4m3 = kFp8;                 // both products on the E4M3 codes
+    constexpr int kNSq = tc_cols_s(G, kE4m3);    // columns of S
+    constexpr int kNSo = tc_cols_o(G, kE4m3);    // columns of O
+    constexpr uint32_t kTmemCols = tc_tmem_cols(kNSq, kNSo);
+    constexpr int kStages = tc_stages(kE4m3);
+    constexpr int kStageBytes = tc_stage_bytes(kE4m3);
+    constexpr TcLayout Lay(G, kE4m3);
     extern __shared__ __align__(1024) unsigned char smem[];
-    unsigned char *k_t = smem + kKOff;
-    unsigned char *v_t = smem + kVOff;
-    unsigned char *q_t = smem + kQOff;
-    unsigned char *p_t = smem + kPOff;
-    float *red = reinterpret_cast<float *>(smem + kRedOff);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
-    uint64_t *k_full = bars + 0, *k_empty = bars + 1, *v_full = bars + 2, *v_empty = bars + 3;
-    uint64_t *s_full = bars + 4, *o_full = bars + 6, *p_full = bars + 8, *q_full = bars + 9;
-    uint64_t *k_stage = bars + 10, *v_stage = bars + 11;  // FP8: codes landed
-    float *qscale = reinterpret_cast<float *>(smem + kQScaleOff);  // kE4m3: logit factor per query row
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMiscOff);
-    int *fail = reinterpret_cast<int *>(smem + kMiscOff + 4);
-    int *lazy_flag = reinterpret_cast<int *>(smem + kMiscOff + 8);  // [4], by chunk & 3
+    unsigned char *k_t = smem + Lay.k_off;
+    unsigned char *v_t = smem + Lay.v_off;
+    unsigned char *q_t = smem + Lay.q_off;
+    unsigned char *p_t = smem + Lay.p_off;
+    float *red = reinterpret_cast<float *>(smem + Lay.red_off);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay.bar_off);
+    uint64_t *k_full = bars + 0, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 6;  // [kStages]
+    uint64_t *s_full = bars + 8, *o_full = bars + 10, *p_full = bars + 12, *q_full = bars + 13;
+    float *qscale = reinterpret_cast<float *>(smem + Lay.qscale_off);  // kE4m3: logit factor per query row
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay.misc_off);
+    int *fail = reinterpret_cast<int *>(smem + Lay.misc_off + 4);
+    int *lazy_flag = reinterpret_cast<int *>(smem + Lay.misc_off + 8);  // [4], by chunk & 3
 
     const int kvh = blockIdx.y;
     // this CTA streams partitions part0 .. part0 + ppc - 1 (those that exist)
@@ -282,6 +247,18 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     pdl_wait();
     const int s = scheduled_seq(p, blockIdx.z, part0 == 0 && kvh == 0 && tid == 0);
     if (s < 0) return;
+    // Without a window a CTA's slice of the table starts at part0 *
+    // part_blocks whatever the context length: the producers issue its first
+    // two windows now, so their latency overlaps the length load and the
+    // set-up below.
+    TablePrefetch pre{false, 0, 0};
+    if ((warp == kWarpK || warp == kWarpV) && p.window <= 0) {
+        const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+        const int bi = part0 * p.part_blocks + lane;
+        pre.valid = true;
+        if (bi < p.max_blocks_per_seq) pre.w0 = row[bi];
+        if (bi + 32 < p.max_blocks_per_seq) pre.w1 = row[bi + 32];
+    }
     // flat q / out row of row r: plain decode keeps the group's rows contiguous
     auto row_of = [&](int r) -> int64_t {
         if constexpr (kMasked) return query_row(p, s, kvh, r);
@@ -320,12 +297,12 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     if (tid == 0) {
         *fail = 0;
         for (int i = 0; i < 4; ++i) lazy_flag[i] = 0;
-        mbar_init(k_full, kFp8 && !kE4m3 ? 32 : 1);  // widened in place: the producer's 32 lanes
-        mbar_init(k_empty, 1);
-        mbar_init(v_full, kFp8 && !kE4m3 ? 32 : 1);
-        mbar_init(v_empty, 1);
-        mbar_init(k_stage, 1);
-        mbar_init(v_stage, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         mbar_init(&o_full[0], 1);
@@ -340,74 +317,68 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpK) {
-        if constexpr (kE4m3)
-            produce_tile<true>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-        else if constexpr (kFp8)
-            produce_tile_fp8(p, &tmap_k, k_t, k_stage, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-        else
-            produce_tile(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        produce_tile<kE4m3, kStages>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane, pre);
     } else if (warp == kWarpV) {
-        if constexpr (kE4m3)
-            produce_tile<true>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-        else if constexpr (kFp8)
-            produce_tile_fp8(p, &tmap_v, v_t, v_stage, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
-        else
-            produce_tile(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane);
+        produce_tile<kE4m3, kStages>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane, pre);
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc_qk =
-                kE4m3 ? tc::instr_desc_e4m3(false, kChunk, kNS) : tc::instr_desc_f16(kBf16, false, kChunk, kN);
+                kE4m3 ? tc::instr_desc_e4m3(false, kChunk, kNSq) : tc::instr_desc_f16(kBf16, false, kChunk, kN);
             constexpr uint32_t idesc_pv =
-                kE4m3 ? tc::instr_desc_e4m3(true, kD, kNS) : tc::instr_desc_f16(kBf16, true, kD, kN);
+                kE4m3 ? tc::instr_desc_e4m3(true, kD, kNSo) : tc::instr_desc_f16(kBf16, true, kD, kN);
             const uint32_t kb = smem_addr(k_t), vb = smem_addr(v_t), qb = smem_addr(q_t), pb = smem_addr(p_t);
             auto pv = [&](int c) -> bool {
-                if (!wait_ok(p_full, c & 1, fail) || !wait_ok(v_full, c & 1, fail)) return false;
+                const int st = c % kStages;
+                if (!wait_ok(p_full, c & 1, fail) || !wait_ok(&v_full[st], (c / kStages) & 1, fail)) return false;
                 tc::fence_after_sync();
+                const uint32_t vs = vb + st * kStageBytes;
                 if constexpr (kE4m3) {
                     // V codes MN-major (a token's 128 dims are one 128-byte atom row),
                     // 32 tokens per MMA; P parts K-major, one 128-byte row per column
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 32; ++kk) {
-                        const uint64_t a = tc::smem_desc(vb + kk * 4096, kRegion, 1024);
+                        const uint64_t a = tc::smem_desc(vs + kk * 4096, kRegion, 1024);
                         const uint64_t b = tc::smem_desc(pb + kk * 32, 16, 1024);
-                        tc::mma_e4m3(tmem + o_col<kNS>(c & 1), a, b, idesc_pv, kk > 0);
+                        tc::mma_e4m3(tmem + o_col<kNSq, kNSo>(c & 1), a, b, idesc_pv, kk > 0);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk) {
-                        const uint64_t a = tc::smem_desc(vb + kk * 2048, kRegion, 1024);
+                        const uint64_t a = tc::smem_desc(vs + kk * 2048, kRegion, 1024);
                         const uint64_t b = tc::smem_desc(pb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-                        tc::mma_f16(tmem + o_col<kNS>(c & 1), a, b, idesc_pv, kk > 0);
+                        tc::mma_f16(tmem + o_col<kNSq, kNSo>(c & 1), a, b, idesc_pv, kk > 0);
                     }
                 }
                 tc::commit(&o_full[c & 1]);
-                tc::commit(v_empty);
+                tc::commit(&v_empty[st]);
                 return true;
             };
             bool ok = wait_ok(q_full, 0, fail);
             for (int c = 0; c < nch && ok; ++c) {
-                ok = wait_ok(k_full, c & 1, fail);
+                const int st = c % kStages;
+                ok = wait_ok(&k_full[st], (c / kStages) & 1, fail);
                 if (!ok) break;
                 tc::fence_after_sync();
+                const uint32_t ks = kb + st * kStageBytes;
                 if constexpr (kE4m3) {
                     // K codes: one 128-byte row per token; Q parts: one 128-byte row per column
 #pragma unroll
                     for (int kk = 0; kk < kD / 32; ++kk) {
-                        const uint64_t a = tc::smem_desc(kb + kk * 32, 16, 1024);
+                        const uint64_t a = tc::smem_desc(ks + kk * 32, 16, 1024);
                         const uint64_t b = tc::smem_desc(qb + kk * 32, 16, 1024);
-                        tc::mma_e4m3(tmem + s_col<kNS>(c & 1), a, b, idesc_qk, kk > 0);
+                        tc::mma_e4m3(tmem + s_col<kNSq, kNSo>(c & 1), a, b, idesc_qk, kk > 0);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint64_t a = tc::smem_desc(kb + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
+                        const uint64_t a = tc::smem_desc(ks + (kk >> 2) * kRegion + (kk & 3) * 32, 16, 1024);
                         const uint64_t b = tc::smem_desc(qb + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-                        tc::mma_f16(tmem + s_col<kNS>(c & 1), a, b, idesc_qk, kk > 0);
+                        tc::mma_f16(tmem + s_col<kNSq, kNSo>(c & 1), a, b, idesc_qk, kk > 0);
                     }
                 }
                 tc::commit(&s_full[c & 1]);
-                tc::commit(k_empty);
+                tc::commit(&k_empty[st]);
                 if (c >= 1) ok = pv(c - 1);
             }
             if (ok) pv(nch - 1);
@@ -416,9 +387,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     } else {
         // ------------------------------ softmax warps ------------------------------
         {
-            // Q tile: rows = the group's query heads (zero rows up to 16),
-            // K-major 128-byte swizzle, two 64-dim regions.  Loaded while the
-            // producers already stream K and V.
+            // Q tile, loaded while the producers already stream K and V.
             const T *q = reinterpret_cast<const T *>(p.q);
             if constexpr (kE4m3) {
                 // Q as E4M3 parts, one warp per query row r, lane l holding
@@ -462,26 +431,17 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                     }
                     if (lane == 0) qscale[r] = finite ? ldexpf(p.scale_log2, -e) : NAN;
                 }
-                for (int r = kQParts * G + warp; r < kNS; r += kSW)  // padding columns
+                for (int r = kQParts * G + warp; r < kNSq; r += kSW)  // padding columns
                     *reinterpret_cast<uint32_t *>(q_t + tc::sw128_offset8(r, 4 * lane)) = 0u;
             } else {
-            for (int i = tid; i < kN * (kD / 8); i += kST) {
-                const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (r < rows) v = *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + c16 * 8);
-                if constexpr (kFp8 && !std::is_same<T, __half>::value) {
-                    // bf16 q -> f16 for the f16 MMA (exact for 2^-14 <= |q| <= 65504)
-                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 f = E::to_float2(w[j]);
-                        const __half2 hh = __floats2half2_rn(f.x, f.y);
-                        w[j] = *reinterpret_cast<const uint32_t *>(&hh);
-                    }
-                    v = make_uint4(w[0], w[1], w[2], w[3]);
+                // rows = the group's query heads (zero rows up to 16), K-major
+                // 128-byte swizzle, two 64-dim regions
+                for (int i = tid; i < kN * (kD / 8); i += kST) {
+                    const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (r < rows) v = *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + c16 * 8);
+                    *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
                 }
-                *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
-            }
             }
             fence_proxy_async_smem();
             mbar_arrive(q_full);
@@ -496,8 +456,8 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
         const int hi0 = L - p.q_len;
         const int lg = 31 - __clz(p.group);
         const int win = p.window > 0 ? p.window : INT_MAX;
-        // E4M3 products: column j of the result = sum over parts k of part
-        // column kG + j / 16^k (Horner from the last part) of the TMEM buffer at taddr
+        // E4M3 products: column c0 + j of the result = sum over parts k of
+        // TMEM column k G + c0 + j divided by 16^k (Horner from the last part)
         auto ld_parts = [&](auto np, uint32_t taddr, float *v) {
             constexpr int NP = decltype(np)::value;
             if constexpr (G == 4) {
@@ -514,7 +474,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 float b[8];
 #pragma unroll
                 for (int k = NP - 1; k >= 0; --k) {
-                    tc::tmem_ld<8>(taddr + 8 * k, b);
+                    tc::tmem_ld<8>(taddr + G * k + c0, b);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) v[j] = k == NP - 1 ? b[j] : fmaf(v[j], 0.0625f, b[j]);
                 }
@@ -534,9 +494,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             tc::fence_after_sync();
             float o[8];
             if constexpr (kE4m3)
-                ld_parts(std::integral_constant<int, kPParts>{}, tmem + lane_base + o_col<kNS>(c & 1), o);
+                ld_parts(std::integral_constant<int, kPParts>{}, tmem + lane_base + o_col<kNSq, kNSo>(c & 1), o);
             else
-                tc::tmem_ld<8>(tmem + lane_base + o_col<kNS>(c & 1) + c0, o);
+                tc::tmem_ld<8>(tmem + lane_base + o_col<kNSq, kNSo>(c & 1) + c0, o);
 #pragma unroll
             for (int j = 0; j < kGT; ++j) acc[j] = fmaf(acc[j], alpha_prev[j], o[j]);
         };
@@ -609,12 +569,12 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             if (ok) {
                 tc::fence_after_sync();
                 float sv[8];
-                const uint32_t sb = tmem + lane_base + s_col<kNS>(c & 1);
+                const uint32_t sb = tmem + lane_base + s_col<kNSq, kNSo>(c & 1);
                 float scl[kGT];
                 if constexpr (kE4m3) {
                     ld_parts(std::integral_constant<int, kQParts>{}, sb, sv);
 #pragma unroll
-                    for (int j = 0; j < kGT; ++j) scl[j] = qscale[j];
+                    for (int j = 0; j < kGT; ++j) scl[j] = qscale[c0 + j];
                 } else {
                     tc::tmem_ld<8>(sb + c0, sv);
 #pragma unroll
@@ -666,7 +626,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                     }
                 }
             }
-            MT pv[kGT];
+            T pv[kGT];
             uint16_t pc[kPParts][kGT / 2];  // E4M3: the weights' parts, two columns per code pair
             if constexpr (kE4m3) {
                 // w = sum over k of part_k / 16^k, part_0 = E4M3(w), part_k = E4M3(16 r_k) with
@@ -696,8 +656,8 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
 #pragma unroll
                 for (int j = 0; j < kGT; ++j) {
                     // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
-                    pv[j] = (kMasked && x[j] == -INFINITY) ? EM::from_float(0.f) : EM::from_float(ex2(x[j] - m[j]));
-                    l[j] += EM::to_float(pv[j]);  // the rounded weight the MMA sees
+                    pv[j] = (kMasked && x[j] == -INFINITY) ? E::from_float(0.f) : E::from_float(ex2(x[j] - m[j]));
+                    l[j] += E::to_float(pv[j]);  // the rounded weight the MMA sees
                 }
             }
             if (cl > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
@@ -707,32 +667,33 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 // Rows of the partial last block past the context come from the
                 // pool and may hold anything (NaN): zero them in the V tile
                 // once it has landed, so 0 * V stays 0 in the PV product.
-                if (wait_ok(v_full, c & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
+                const int st = c % kStages;
+                unsigned char *vt = v_t + st * kStageBytes;
+                if (wait_ok(&v_full[st], (c / kStages) & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
 #pragma unroll
                     for (int j = 0; j < (kE4m3 ? 1 : 2); ++j)  // E4M3: a token's codes are one 128-byte row
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
-                            *reinterpret_cast<uint4 *>(v_t + j * kRegion + t * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(vt + j * kRegion + t * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            // P tile: K-major, rows = heads, columns = tokens (two 64-token
-            // regions); this thread writes rows c0 .. c0 + (16 / (kSW / 4)) - 1
-            // (its columns, then zero rows up to 16)
+            // P tile: K-major, rows = columns of O, 128-byte rows of tokens
             if constexpr (kE4m3) {
-                // E4M3 part tile: part k of column j in row k G + j, one 128-byte
-                // row of tokens each
+                // E4M3 part tile: part k of column c0 + j in row k G + c0 + j
 #pragma unroll
                 for (int k = 0; k < kPParts; ++k)
 #pragma unroll
                     for (int j = 0; j < kGT; ++j)
-                        p_t[tc::sw128_offset8(k * G + j, t)] = (unsigned char)(pc[k][j / 2] >> (8 * (j & 1)));
+                        p_t[tc::sw128_offset8(k * G + c0 + j, t)] = (unsigned char)(pc[k][j / 2] >> (8 * (j & 1)));
             } else {
+                // two 64-token regions; this thread writes rows c0 .. c0 +
+                // (16 / (kSW / 4)) - 1 (its columns, then zero rows up to 16)
                 unsigned char *pr = p_t + (t >> 6) * (kN * 128);
                 constexpr int kRowsW = kN / (kSW / 4);
 #pragma unroll
                 for (int j = 0; j < kRowsW; ++j) {
-                    const MT v = j < kGT ? pv[j < kGT ? j : 0] : EM::from_float(0.f);
-                    *reinterpret_cast<MT *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
+                    const T v = j < kGT ? pv[j < kGT ? j : 0] : E::from_float(0.f);
+                    *reinterpret_cast<T *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
                 }
             }
             fence_proxy_async_smem();
@@ -772,9 +733,8 @@ EncodeTiledFn encode_fn() {
 // A cache [NB, Hk, 16, 128] seen as rows of 128 elements; boxes of 16 rows
 // x 64 elements with the 128-byte swizzle; out-of-range rows read as zero.
 // An FP8 cache [NB, Hk, 16, 128] seen as rows of 128 one-byte codes; boxes
-// of 16 rows x 128 bytes, unswizzled where the producer converts them,
-// with the 128-byte swizzle where the MMA reads them.
-bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows, bool swizzle) {
+// of 16 rows x 128 bytes with the 128-byte swizzle the MMA reads.
+bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
@@ -782,7 +742,7 @@ bool encode_code_map(CUtensorMap *map, const void *base, int64_t rows, bool swiz
     const cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kBlock};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -804,25 +764,19 @@ template <typename T, int G, bool kMasked, bool kFp8 = false>
 cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
     CUtensorMap tk, tv;
-    const bool ok = kFp8 ? encode_code_map(&tk, p.k_cache, rows, G <= 8) && encode_code_map(&tv, p.v_cache, rows, G <= 8)
+    const bool ok = kFp8 ? encode_code_map(&tk, p.k_cache, rows) && encode_code_map(&tv, p.v_cache, rows)
                          : encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) &&
                                encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = decode_tc_kernel<T, G, kMasked, kFp8>;
-    static int configured[kMaxDevices] = {};
-    static int carveout_set[kMaxDevices] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && !carveout_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        carveout_set[dev] = 1;
-    }
-    e = ensure_smem(kern, kSmemTc, configured);
+    static FuncAttrCache attrs;
+    constexpr int kSmem = TcLayout(G, kFp8).bytes;
+    static_assert(kSmem * tc_ctas_per_sm(G) + 1024 * tc_ctas_per_sm(G) <= 228 * 1024,
+                  "the CTAs per SM must fit in shared memory");
+    cudaError_t e = ensure_smem(kern, kSmem, attrs, /*max_carveout=*/true);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, p.num_kv_heads, p.num_seqs),
-                   dim3(tc_threads(G)), kSmemTc, stream, p, tk, tv,
+                   dim3(tc_threads(G)), kSmem, stream, p, tk, tv,
                    (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);

@@ -129,6 +129,57 @@ def test_fp8_group_sizes_and_head_dims(orc, dtype, D, g):
         compare(out, ref, dtype, f"fp8 g={g} D={D} P={P}")
 
 
+@pytest.mark.parametrize("shift", [20, -30])
+@pytest.mark.parametrize("g,q_len", [(4, 1), (8, 1), (16, 1), (4, 4)])
+def test_fp8_bf16_q_beyond_f16_range(orc, shift, g, q_len):
+    """bf16 queries whose every element lies above f16's largest finite value
+    (magnitudes in [0.5, 1) x 2^20) or below its smallest normal (x 2^-30),
+    with the softmax scale divided by the same power of two so the logits
+    are those of O(1) queries.  The tensor-core FP8 products carry q as E4M3
+    parts under a per-row power of two, so such a q must give the oracle's
+    result on every row count: groups 4, 8, 16 and group 4 x 4 query tokens
+    (16 columns, pa_decode_ext)."""
+    from paged_kv_cache_424_b200 import binding as pa
+    rng = np.random.default_rng(600 + 10 * g + q_len + shift)
+    Hk, D = 2, 128
+    H = Hk * g
+    lens = np.array([q_len, 17, 250, 1100], np.int32)
+    S, MB = len(lens), 72
+    NB = S * MB + 8
+    kc, vc = random_codes(rng, (NB, Hk, 16, D)), random_codes(rng, (NB, Hk, 16, D))
+    tables = rng.permutation(NB)[:S * MB].reshape(S, MB).astype(np.int32)
+    mag = rng.random((S, q_len, H, D), dtype=np.float32) * 0.5 + 0.5
+    sign = np.where(rng.random((S, q_len, H, D)) < 0.5, -1.0, 1.0).astype(np.float32)
+    q4 = torch.from_numpy(mag * sign * np.float32(2.0 ** shift)).cuda().to(torch.bfloat16)
+    qa = q4.float().abs()
+    assert bool((qa > 65504).all()) if shift > 0 else bool((qa < 2.0 ** -14).all() and (qa > 0).all())
+    qbits = q4.view(torch.int16).cpu().numpy().view(np.uint16)
+    ks, vs = float(np.float32(0.09)), float(np.float32(0.13))
+    scale = float(np.float32(np.float32(1 / np.sqrt(D)) * np.float32(2.0 ** -shift)))
+    dk, dv = torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda()
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    maxlen = int(lens.max())
+    if q_len == 1:
+        ref = orc.paged_decode_fp8(qbits[:, 0], kc, vc, tables, lens, scale, ks, vs, "bf16")
+        q = q4[:, 0].contiguous()
+    else:
+        ref = orc.paged_decode_ext(qbits, kc, vc, tables, lens, scale, "bf16", q_len, 0, ks, vs)
+        q = q4
+    for P in (0, 16):
+        out = torch.full_like(q, float("nan"))
+        if q_len == 1:
+            n = pa.pa_decode_workspace_size(pa.dims_of(q, dk, bt), maxlen, P)
+            ws = torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
+            pa.pa_decode_fp8(out, q, dk, dv, bt, cl, scale, ks, vs, Hk, maxlen, P, ws)
+        else:
+            opts = pa.pa_decode_opts(q_len, 0, ks, vs)
+            n = pa.pa_decode_ext_workspace_size(pa.ext_dims(q, dk, bt), opts, maxlen, P)
+            ws = torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
+            pa.pa_decode_ext(out, q, dk, dv, bt, cl, scale, Hk, maxlen, q_len, 0, ks, vs, P, ws)
+        torch.cuda.synchronize()
+        compare(out, ref, "bf16", f"fp8 bf16 q x 2^{shift} g={g} q_len={q_len} P={P}")
+
+
 # ---------------------------------------------------------------------------
 # decode over FP8 caches: the workloads at reduced and full sizes
 # ---------------------------------------------------------------------------

@@ -6,12 +6,15 @@ inside a framework whose memory pool it may not touch, or a path where
 cudaMalloc's implicit synchronisation is not acceptable.  pa_decode_noalloc
 takes no workspace and uses the library's own 64 MiB static device scratch.
 
-These tests call it through the C ABI and check that its output matches
-pa_decode (with a caller workspace) within the parity tolerances, on two
-calls in a row with different shapes (the second call finds the first
-call's data still in the shared scratch), and that a plan needing more than
-the scratch holds is refused before anything is enqueued.  This file is
-collected last so that a stop-at-first-failure run has run everything else.
+These tests call it through the C ABI, on two calls in a row with different
+shapes (the second call finds the first call's data still in the shared
+scratch).  Each output must equal pa_decode's (with a caller workspace) bit
+for bit, since both run the same plan through the same kernels and only the
+scratch's address differs, so a stale partial or a wrong offset cannot hide
+under a tolerance; and it must match the CPU oracle within the parity
+tolerances.  A plan needing more than the scratch holds is refused before
+anything is enqueued.  This file is collected last so that a
+stop-at-first-failure run has run everything else.
 """
 import numpy as np
 import pytest
@@ -54,14 +57,16 @@ def _both(p: Paged, scale: float, P: int):
     return got, ref
 
 
-def test_noalloc_matches_pa_decode_two_calls_in_a_row():
+def test_noalloc_matches_pa_decode_two_calls_in_a_row(orc):
     rng = np.random.default_rng(2024)
     first = Paged(rng, [3000, 17, 1200, 4097], 32, 8, 128, "bf16")
     got, ref = _both(first, 0.088, 0)
-    compare(got, ref.double().cpu().numpy(), "bf16", "noalloc call 1")
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), "call 1: differs from pa_decode"
+    compare(got, first.run(orc, 0.088), "bf16", "noalloc call 1 vs the oracle")
     second = Paged(rng, [700, 2500, 33], 16, 16, 64, "f16")
     got, ref = _both(second, 0.125, 16)
-    compare(got, ref.double().cpu().numpy(), "f16", "noalloc call 2")
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), "call 2: differs from pa_decode"
+    compare(got, second.run(orc, 0.125), "f16", "noalloc call 2 vs the oracle")
 
 
 def test_noalloc_refuses_a_plan_larger_than_its_scratch():
