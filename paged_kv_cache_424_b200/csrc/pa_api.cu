@@ -107,13 +107,29 @@ int sm_count() {
 // 0.78 of the copy roofline against 0.87 at 1024), as long as the grid
 // keeps at least two waves of resident CTAs.  Each partition still gets its
 // own partial and the merge is unchanged.
-int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows) {
+int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows, bool fp8) {
     if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= 64) return 1;
-    const int64_t slots = (int64_t)sm_count() * (rows > 8 ? 2 : 3);
+    const int64_t slots = (int64_t)sm_count() * (rows > 8 || fp8 ? 2 : 3);  // resident CTAs per SM
     const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
     int ppc = 64 / pl.part_blocks;
     while (ppc > 1 && pairs * ((pl.max_parts + ppc - 1) / ppc) < 2 * slots) ppc >>= 1;
     return ppc;
+}
+
+// KV heads one tensor-core CTA streams back to back (plain decode only: the
+// query rows of two heads of a group of 4 or 8 fit the Q tile's 16 rows).
+// Short sequences give CTAs of a few chunks, each paying the set-up and the
+// first loads' latency (measured: 1 chunk per CTA ran at 0.72 of the
+// throughput of 8); two heads per CTA halve that count.  Only with
+// 1024-token partitions or a single one (a CTA then streams at most 16
+// chunks) and while the grid keeps two waves of resident CTAs.
+int tc_heads_per_cta(const Plan &pl, const pa_dims *d, int rows, bool plain) {
+    if (!plain || (pl.max_parts > 1 && pl.part_blocks < 64) || pl.part_blocks > 64) return 1;
+    const int64_t slots = (int64_t)sm_count() * 3;
+    int hpc = 1;
+    if (2 * rows <= 16 && d->num_kv_heads % 2 == 0 && (int64_t)d->num_seqs * (d->num_kv_heads / 2) >= 2 * slots)
+        hpc = 2;
+    return hpc;
 }
 
 pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
@@ -198,9 +214,12 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.seq_order = seq_order;
     const int rows = row_capacity(g * q_len);
     const int tc = tc_rows(dims, rows);
-    p.parts_per_cta = tc ? tc_parts_per_cta(pl, dims->num_seqs, dims->num_kv_heads, tc) : 1;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_fp8(dims);
+    p.parts_per_cta = tc ? tc_parts_per_cta(pl, dims->num_seqs, dims->num_kv_heads, tc, fp8) : 1;
+    // the plain tensor-core variant: one query token, no window, unscaled 16-bit V
+    const bool plain = tc && !fp8 && q_len == 1 && window == 0 && v_scale == 1.f;
+    p.heads_per_cta = plain && p.parts_per_cta == 1 ? tc_heads_per_cta(pl, dims, tc, true) : 1;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e = tc ? pa::launch_decode_tc(p, dims->dtype, tc, fp8, cs)
                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, rows, fp8, cs);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "pa_decode_fp8 launch" : "pa_decode launch");

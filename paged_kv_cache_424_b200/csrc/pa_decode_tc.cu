@@ -9,8 +9,8 @@
 //   O^T (128 dims x 16)  = V^T (128 x 128 tokens) . P^T (128 x 16)  [PV]
 // (the G query rows padded to the MMA's N = 16).
 //
-// CTA = (partition, KV head, sequence): 7 warps (11 with 16 columns, whose
-// softmax work is split over 8 warps, 8 columns each).
+// CTA = (partition, KV head, sequence): 8 warps (12 with 16 columns, whose
+// softmax work is split over 8 warps, 8 columns each); the last warp idles.
 //   warp 4  K producer and warp 6  V producer (8 and 10 with 16 columns): per chunk, 2-D tiled TMA loads
 //           of the 8 blocks' K (or V) rows (16 rows x 64 dims per box,
 //           128-byte swizzle) into the K (or V) tile, as soon as the previous
@@ -80,25 +80,29 @@ __device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)((2 + b) * t
 static_assert(tc_tmem_cols(16, 16) == 64 && tc_tmem_cols(32, 32) == 128 && tc_tmem_cols(48, 64) == 256,
               "TMEM columns per CTA");
 
-// K / V stages: a 16-bit chunk fills its 32 KiB tile area (two 64-dim
-// regions), one stage; E4M3 codes take 16 KiB, so each area holds two
-// stages and the loads of chunk c + 1 overlap the products of chunk c.
-__host__ __device__ constexpr int tc_stages(bool e4m3) { return e4m3 ? 2 : 1; }
+// K / V stages: a 16-bit chunk fills a 32 KiB tile area (two 64-dim
+// regions), one stage per operand at 3 CTAs per SM; E4M3 codes take 16 KiB
+// a chunk, three stages per operand at 2 CTAs per SM, so the loads of the
+// next chunks overlap the products and the softmax of the current one.
+constexpr int kMaxStages = 3;
+__host__ __device__ constexpr int tc_stages(bool e4m3) { return e4m3 ? 3 : 1; }
 __host__ __device__ constexpr int tc_stage_bytes(bool e4m3) { return e4m3 ? kRegion : 2 * kRegion; }
 
 // Shared-memory layout (bytes from the 1024-aligned base): K tile area,
 // V tile area, Q tile (16-bit: two 64-dim regions of 16 rows; E4M3: NSq
 // rows of 128 codes), P tile (16-bit: two 64-token regions of 16 rows;
-// E4M3: NSo rows of 128 codes), the cross-warp reduction [2][4][16] floats,
-// the mbarriers, TMEM base / fail flag / 4 lazy-max flags, and the per-row
-// logit factors of the E4M3 path.
-constexpr int kNumBars = 16;
+// E4M3: NSo rows of 128 codes), the cross-warp reduction [2][4][16]
+// floats, the mbarriers, TMEM base / fail flag / 4 lazy-max flags, and the
+// per-row logit factors of the E4M3 path.
+constexpr int kNumBars = 4 * kMaxStages + 6;
 struct TcLayout {
     int k_off, v_off, q_off, p_off, red_off, bar_off, misc_off, qscale_off, bytes;
     __host__ __device__ constexpr TcLayout(int G, bool e4m3)
-        : k_off(0), v_off(2 * kRegion), q_off(4 * kRegion), p_off(q_off + (e4m3 ? tc_cols_s(G, true) * 128 : 2 * kN * 128)),
+        : k_off(0), v_off(tc_stages(e4m3) * tc_stage_bytes(e4m3)), q_off(2 * tc_stages(e4m3) * tc_stage_bytes(e4m3)),
+          p_off(q_off + (e4m3 ? tc_cols_s(G, true) * 128 : 2 * kN * 128)),
           red_off(p_off + (e4m3 ? tc_cols_o(G, true) * 128 : 2 * kN * 128)), bar_off(red_off + 2 * 4 * kN * 4),
-          misc_off(bar_off + kNumBars * 8), qscale_off(misc_off + 32), bytes(qscale_off + kN * 4) {}
+          misc_off(bar_off + kNumBars * 8), qscale_off(misc_off + 32),
+          bytes(qscale_off + kN * 4) {}
 };
 
 __device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
@@ -136,43 +140,47 @@ struct TablePrefetch {
     int32_t w0, w1;
 };
 
-template <bool kCodes, int kStages>
+template <bool kCodes, int kStages, int nheads>
 __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtensorMap *tmap, unsigned char *tile,
-                                             uint64_t *full, uint64_t *empty, int *fail, int s, int kvh, int b0,
+                                             uint64_t *full, uint64_t *empty, int *fail, int s, int kvh0, int b0,
                                              int nb, int nch, int oob_row, int lane, const TablePrefetch &pre) {
     constexpr int kStageBytes = tc_stage_bytes(kCodes);
     const int32_t *row = p.block_tables + (int64_t)s * p.max_blocks_per_seq + b0;
-    auto slot_of = [&](int bi, int32_t entry) -> int {
+    auto slot_of = [&](int bi, int32_t entry, int kvh) -> int {
         return bi < nb ? (int)((checked_block(p, entry) * p.num_kv_heads + kvh) * kBlock) : oob_row;
     };
-    auto window = [&](int w) -> int {
+    auto window = [&](int w, int kvh) -> int {
         const int bi = w * 32 + lane;
-        return slot_of(bi, bi < nb ? row[bi] : 0);
+        return slot_of(bi, bi < nb ? row[bi] : 0, kvh);
     };
     if (lane == 0) prefetch_tmap(tmap);
-    int cur = pre.valid ? slot_of(lane, pre.w0) : window(0);
-    int next = nb > 32 ? (pre.valid ? slot_of(32 + lane, pre.w1) : window(1)) : oob_row;
-    int issued = 0;
-    for (int c = 0; c < nch; ++c) {
-        if (c > 0 && (c & 3) == 0) {
-            cur = next;
-            next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1) : oob_row;
+    int issued = 0;  // chunks issued, counted over all heads (stages and phases follow this count)
+    bool ok = true;
+    for (int h = 0; h < nheads && ok; ++h) {
+        const int kvh = kvh0 + h;
+        int cur = pre.valid ? slot_of(lane, pre.w0, kvh) : window(0, kvh);
+        int next = nb > 32 ? (pre.valid ? slot_of(32 + lane, pre.w1, kvh) : window(1, kvh)) : oob_row;
+        for (int c = 0; c < nch; ++c) {
+            if (c > 0 && (c & 3) == 0) {
+                cur = next;
+                next = (c / 4 + 1) * 32 < nb ? window(c / 4 + 1, kvh) : oob_row;
+            }
+            const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
+            const int cc = issued;
+            const int st = cc % kStages;
+            if (lane == 0) {
+                ok = cc < kStages || wait_ok(&empty[st], (cc / kStages - 1) & 1, fail);
+                if (ok) mbar_arrive_expect_tx(&full[st], kCodes ? kRegion : 2 * kRegion);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            unsigned char *dst = tile + st * kStageBytes;
+            if (lane < kChunkBlocks) {
+                tc::tma_load_2d(dst + lane * 2048, tmap, 0, y, &full[st]);
+                if constexpr (!kCodes) tc::tma_load_2d(dst + kRegion + lane * 2048, tmap, 64, y, &full[st]);
+            }
+            issued = cc + 1;
         }
-        const int y = __shfl_sync(0xffffffffu, cur, ((c & 3) << 3) + (lane & 7));
-        const int st = c % kStages;
-        bool ok = true;
-        if (lane == 0) {
-            ok = c < kStages || wait_ok(&empty[st], (c / kStages - 1) & 1, fail);
-            if (ok) mbar_arrive_expect_tx(&full[st], kCodes ? kRegion : 2 * kRegion);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        unsigned char *dst = tile + st * kStageBytes;
-        if (lane < kChunkBlocks) {
-            tc::tma_load_2d(dst + lane * 2048, tmap, 0, y, &full[st]);
-            if constexpr (!kCodes) tc::tma_load_2d(dst + kRegion + lane * 2048, tmap, 64, y, &full[st]);
-        }
-        issued = c + 1;
     }
     // After a failure the last chunks issued may still be landing (their
     // consumer gave up): give each a bounded chance before the CTA exits.
@@ -185,14 +193,21 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
 
 // Softmax warps: one per TMEM lane quadrant, each thread holding the state
 // of every column; with 16 columns two warps per quadrant, each owning 8 of
-// the columns, so a thread's state stays that of 8 columns.  Then the K
-// producer, the MMA issuer and the V producer.
-__host__ __device__ constexpr int tc_soft_warps(int G) { return G > 8 ? 8 : 4; }
-__host__ __device__ constexpr int tc_threads(int G) { return (tc_soft_warps(G) + 3) * 32; }
+// the columns, so a thread's state stays that of 8 columns.  Then one more
+// group of 4 warps: the K producer, the MMA issuer, the V producer and an
+// idle warp.  The compiler caps registers as if a CTA's warps came in fours
+// anyway (80 per thread for 3 CTAs of 7 or 8 warps per SM); with the fourth
+// warp present it spills far less in the softmax loop (measured with
+// -Xptxas -v: 44 -> 4 bytes for 8 columns).
+// FP8 caches: 8 softmax warps whatever the group, two per quadrant, each
+// thread holding half the columns (the E4M3 weight split is the per-chunk
+// work that sets the pace there).
+__host__ __device__ constexpr int tc_soft_warps(int G, bool e4m3) { return G > 8 || e4m3 ? 8 : 4; }
+__host__ __device__ constexpr int tc_threads(int G, bool e4m3) { return (tc_soft_warps(G, e4m3) + 4) * 32; }
 
 // CTAs per SM: 3 (registers and shared memory both allow it) except with 16
 // columns, whose 11 warps fit twice.
-__host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; }
+__host__ __device__ constexpr int tc_ctas_per_sm(int G, bool e4m3) { return G > 8 || e4m3 ? 2 : 3; }
 
 // G: columns of S (query rows per KV head: the group, or group x query
 // tokens with kMasked, padded to a power of two).
@@ -203,16 +218,19 @@ __host__ __device__ constexpr int tc_ctas_per_sm(int G) { return G > 8 ? 2 : 3; 
 // finite 16-bit q to within 2^-15 of the row's largest |q|), P into four
 // parts (|w - sum| <= 2^-12 w + 2^-22); the f32 products of the parts are
 // recombined when S and O are read from TMEM.
-template <typename T, int G, bool kMasked, bool kFp8>
-__global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
+// kHpc: KV heads one CTA streams (2 only for plain 16-bit decode with G * 2
+// <= 16 query rows; with 1 the head bookkeeping compiles away).
+template <typename T, int G, bool kMasked, bool kFp8, int kHpc = 1>
+__global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const int oob_row) {
     static_assert(!kFp8 || kMasked, "FP8 launches take the masked variant (it applies v_scale)");
+    static_assert(kHpc == 1 || (!kMasked && G * kHpc <= kN), "several heads per CTA: plain decode, 16 rows");
     using E = Elem<T>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    constexpr int kSW = tc_soft_warps(G);       // softmax warps
+    constexpr int kSW = tc_soft_warps(G, kFp8);  // softmax warps
     constexpr int kST = kSW * 32;                // softmax threads
-    constexpr int kGT = G > 8 ? 8 : G;           // columns per softmax thread
+    constexpr int kGT = kFp8 ? G / 2 : G > 8 ? 8 : G;  // columns per softmax thread
     constexpr int kWarpK = kSW, kWarpMma = kSW + 1, kWarpV = kSW + 2;
     constexpr bool kE4m3 = kFp8;                 // both products on the E4M3 codes
     constexpr int kNSq = tc_cols_s(G, kE4m3);    // columns of S
@@ -228,16 +246,20 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     unsigned char *p_t = smem + Lay.p_off;
     float *red = reinterpret_cast<float *>(smem + Lay.red_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay.bar_off);
-    uint64_t *k_full = bars + 0, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 6;  // [kStages]
-    uint64_t *s_full = bars + 8, *o_full = bars + 10, *p_full = bars + 12, *q_full = bars + 13;
+    uint64_t *k_full = bars, *k_empty = bars + kMaxStages;  // [kStages]
+    uint64_t *v_full = bars + 2 * kMaxStages, *v_empty = bars + 3 * kMaxStages;
+    uint64_t *s_full = bars + 4 * kMaxStages, *o_full = s_full + 2, *p_full = s_full + 4, *q_full = s_full + 5;
     float *qscale = reinterpret_cast<float *>(smem + Lay.qscale_off);  // kE4m3: logit factor per query row
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay.misc_off);
     int *fail = reinterpret_cast<int *>(smem + Lay.misc_off + 4);
     int *lazy_flag = reinterpret_cast<int *>(smem + Lay.misc_off + 8);  // [4], by chunk & 3
 
-    const int kvh = blockIdx.y;
-    // this CTA streams partitions part0 .. part0 + ppc - 1 (those that exist)
-    // back to back: one set-up, one pipeline, one partial per partition
+    // this CTA streams KV heads kvh .. kvh + hpc - 1 (plain decode only: the
+    // query rows of hpc heads, G each, fill the Q tile's 16 rows) and, for
+    // each, partitions part0 .. part0 + ppc - 1 (those that exist), back to
+    // back: one set-up, one pipeline, one partial per (head, partition)
+    constexpr int hpc = kHpc;
+    const int kvh = blockIdx.y * hpc;
     const int ppc = p.parts_per_cta;
     const int part0 = blockIdx.x * ppc;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -245,7 +267,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     T *out = reinterpret_cast<T *>(p.out);
     pdl_launch_dependents();
     pdl_wait();
-    const int s = scheduled_seq(p, blockIdx.z, part0 == 0 && kvh == 0 && tid == 0);
+    const int s = scheduled_seq(p, blockIdx.z, part0 == 0 && blockIdx.y == 0 && tid == 0);
     if (s < 0) return;
     // Without a window a CTA's slice of the table starts at part0 *
     // part_blocks whatever the context length: the producers issue its first
@@ -264,9 +286,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
         if constexpr (kMasked) return query_row(p, s, kvh, r);
         return (int64_t)s * H + head0 + r;
     };
-    const int rows = kMasked ? p.group * p.q_len : G;
+    const int rows = kMasked ? p.group * p.q_len : G * hpc;  // real Q rows of the CTA
 
-    const SeqSplit sp = seq_split(p, s, part0 == 0 && kvh == 0 && tid == 0);
+    const SeqSplit sp = seq_split(p, s, part0 == 0 && blockIdx.y == 0 && tid == 0);
     const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part0 >= nparts) return;
     const int nmine = min(ppc, nparts - part0);  // partitions of this CTA
@@ -288,6 +310,7 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     const int cpp = ppc > 1 ? p.part_blocks / kChunkBlocks : nch;
     const int tok0 = b0 * kBlock;
     const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
+    const int nct = hpc * nch;                              // chunks of all the CTA's heads
 
     // ---- set-up -----------------------------------------------------------------
     if (warp == kWarpMma) {
@@ -317,9 +340,11 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpK) {
-        produce_tile<kE4m3, kStages>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row, lane, pre);
+        produce_tile<kE4m3, kStages, kHpc>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row,
+                                           lane, pre);
     } else if (warp == kWarpV) {
-        produce_tile<kE4m3, kStages>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row, lane, pre);
+        produce_tile<kE4m3, kStages, kHpc>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row,
+                                           lane, pre);
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
@@ -328,9 +353,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             constexpr uint32_t idesc_pv =
                 kE4m3 ? tc::instr_desc_e4m3(true, kD, kNSo) : tc::instr_desc_f16(kBf16, true, kD, kN);
             const uint32_t kb = smem_addr(k_t), vb = smem_addr(v_t), qb = smem_addr(q_t), pb = smem_addr(p_t);
-            auto pv = [&](int c) -> bool {
+            // PV(c): O^T = V^T . P^T into O buffer c & 1
+            auto issue_pv = [&](int c) {
                 const int st = c % kStages;
-                if (!wait_ok(p_full, c & 1, fail) || !wait_ok(&v_full[st], (c / kStages) & 1, fail)) return false;
                 tc::fence_after_sync();
                 const uint32_t vs = vb + st * kStageBytes;
                 if constexpr (kE4m3) {
@@ -352,13 +377,10 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 }
                 tc::commit(&o_full[c & 1]);
                 tc::commit(&v_empty[st]);
-                return true;
             };
-            bool ok = wait_ok(q_full, 0, fail);
-            for (int c = 0; c < nch && ok; ++c) {
+            // S(c) = K . Q^T into S buffer c & 1
+            auto issue_s = [&](int c) {
                 const int st = c % kStages;
-                ok = wait_ok(&k_full[st], (c / kStages) & 1, fail);
-                if (!ok) break;
                 tc::fence_after_sync();
                 const uint32_t ks = kb + st * kStageBytes;
                 if constexpr (kE4m3) {
@@ -379,12 +401,44 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 }
                 tc::commit(&s_full[c & 1]);
                 tc::commit(&k_empty[st]);
-                if (c >= 1) ok = pv(c - 1);
+            };
+            // The two products are issued in whichever order their inputs
+            // arrive, polled without blocking: S(n) once K(n) has landed and
+            // PV(n - 2) is issued (S(n) reuses the TMEM buffer of S(n - 2),
+            // which the softmax warps read before handing over P(n - 2));
+            // PV(n) once P(n) and V(n) are there.  A late K never holds back
+            // a ready PV, nor a late P a ready S.  Bounded like every wait.
+            bool ok = wait_ok(q_full, 0, fail);
+            int ns = 0, npv = 0;
+            long long t_last = clock64();
+            while (ok && npv < nct) {
+                bool progress = false;
+                if (ns < nct && ns <= npv + 1 && mbar_test(&k_full[ns % kStages], (ns / kStages) & 1)) {
+                    issue_s(ns);
+                    ++ns;
+                    progress = true;
+                }
+                if (npv < ns && mbar_test(p_full, npv & 1) &&
+                    mbar_test(&v_full[npv % kStages], (npv / kStages) & 1)) {
+                    issue_pv(npv);
+                    ++npv;
+                    progress = true;
+                }
+                if (progress) {
+                    t_last = clock64();
+                } else if (is_failed(fail)) {
+                    ok = false;
+                } else if (clock64() - t_last > kWaitLimitCycles) {
+                    flag_error(PA_DEVERR_TIMEOUT);
+                    atomicOr(fail, 1);
+                    ok = false;
+                } else {
+                    __nanosleep(32);
+                }
             }
-            if (ok) pv(nch - 1);
         }
         __syncwarp();
-    } else {
+    } else if (warp < kSW) {
         // ------------------------------ softmax warps ------------------------------
         {
             // Q tile, loaded while the producers already stream K and V.
@@ -464,19 +518,19 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 float t16[16];
                 tc::tmem_ld<16>(taddr, t16);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float a = t16[(NP - 1) * 4 + j];
+                for (int j = 0; j < kGT; ++j) {
+                    float a = t16[(NP - 1) * 4 + c0 + j];
 #pragma unroll
-                    for (int k = NP - 2; k >= 0; --k) a = fmaf(a, 0.0625f, t16[k * 4 + j]);
+                    for (int k = NP - 2; k >= 0; --k) a = fmaf(a, 0.0625f, t16[k * 4 + c0 + j]);
                     v[j] = a;
                 }
             } else {
-                float b[8];
+                float b[kGT];
 #pragma unroll
                 for (int k = NP - 1; k >= 0; --k) {
-                    tc::tmem_ld<8>(taddr + G * k + c0, b);
+                    tc::tmem_ld<kGT>(taddr + G * k + c0, b);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) v[j] = k == NP - 1 ? b[j] : fmaf(v[j], 0.0625f, b[j]);
+                    for (int j = 0; j < kGT; ++j) v[j] = k == NP - 1 ? b[j] : fmaf(v[j], 0.0625f, b[j]);
                 }
             }
         };
@@ -489,22 +543,28 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             acc[j] = 0.f;
             alpha_prev[j] = 1.f;
         }
-        auto epilogue = [&](int c) {
-            if (!wait_ok(&o_full[c & 1], (c >> 1) & 1, fail)) return;
+        auto wait_o = [&](int c) { return wait_ok(&o_full[c & 1], (c >> 1) & 1, fail); };
+        // O of chunk c (CTA-wide chunk count) of the head whose query rows
+        // start at Q-tile row hgc
+        auto load_o = [&](int c, int hgc) {
             tc::fence_after_sync();
             float o[8];
             if constexpr (kE4m3)
                 ld_parts(std::integral_constant<int, kPParts>{}, tmem + lane_base + o_col<kNSq, kNSo>(c & 1), o);
             else
-                tc::tmem_ld<8>(tmem + lane_base + o_col<kNSq, kNSo>(c & 1) + c0, o);
+                tc::tmem_ld<kGT>(tmem + lane_base + o_col<kNSq, kNSo>(c & 1) + hgc + c0, o);
 #pragma unroll
             for (int j = 0; j < kGT; ++j) acc[j] = fmaf(acc[j], alpha_prev[j], o[j]);
         };
+        auto epilogue = [&](int c, int hgc) {
+            if (wait_o(c)) load_o(c, hgc);
+        };
         const bool has_tail = (b0 + nb == nblk) && (L % kBlock) != 0;  // partial last block here
-        // the partial of partition part0 + pi: per-column sums over the 4
-        // lane quadrants, then o = acc / l (and lse) to the output or the
-        // workspace; the last sync frees `red` for the next chunk's maxima
-        auto finalize = [&](int pi) {
+        // the partial of partition part0 + pi of head kvh + hh: per-column
+        // sums over the 4 lane quadrants, then o = acc / l (and lse) to the
+        // output or the workspace; the last sync frees `red` for the next
+        // chunk's maxima (fewer syncs made the compiler spill in the loop)
+        auto finalize = [&](int hh, int pi) {
             float *rl = red;
             softmax_sync<kST>();
 #pragma unroll
@@ -535,10 +595,11 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                         }
                     } else {  // plain decode: every column has tokens, V unscaled
                         const float o = acc[j] / lt;
+                        const int64_t qh = (int64_t)s * H + head0 + hh * G + h;  // query head of column h
                         if (direct) {
-                            out[((int64_t)s * H + head0 + h) * kD + t] = E::from_float(o);
+                            out[qh * kD + t] = E::from_float(o);
                         } else {
-                            const int64_t r = ((int64_t)s * H + head0 + h) * p.max_parts + part;
+                            const int64_t r = qh * p.max_parts + part;
                             p.ws_o[r * kD + t] = o;
                             if (t == 0) p.ws_lse[r] = m[j] + log2f(lt);
                         }
@@ -547,14 +608,24 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             }
             softmax_sync<kST>();
         };
-        for (int c = 0; c < nch; ++c) {
+        int hh = 0, cbase = 0;  // the head of chunk cc, and the CTA-wide index of its first chunk
+        for (int cc = 0; cc < nct; ++cc) {
             float x[kGT];
+            if constexpr (kHpc > 1) {
+                if (cc - cbase == nch) {
+                    cbase += nch;
+                    ++hh;
+                }
+            }
+            const int c = cc - cbase;  // this head's chunk
+            const int hg = hh * G;     // its first query row in the Q tile
             const int tok = tok0 + c * kChunk + t;
             const int cl = c % cpp;  // chunk index within its partition
-            if (cl == 0 && c > 0) {
-                // chunk c - 1 closed a partition: finish and write it, start afresh
-                epilogue(c - 1);
-                finalize(c / cpp - 1);
+            if (cl == 0 && cc > 0) {
+                // chunk cc - 1 closed a partition (or a head): finish and write it, start afresh
+                const int hp = c == 0 ? hh - 1 : hh;
+                epilogue(cc - 1, hp * G);
+                finalize(hp, c == 0 ? (nch - 1) / cpp : c / cpp - 1);
 #pragma unroll
                 for (int j = 0; j < kGT; ++j) {
                     m[j] = -INFINITY;
@@ -564,19 +635,19 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                 }
             }
             const bool valid = tok < tok_end;
-            bool ok = wait_ok(&s_full[c & 1], (c >> 1) & 1, fail);
+            bool ok = wait_ok(&s_full[cc & 1], (cc >> 1) & 1, fail);
             bool exceed = false;
             if (ok) {
                 tc::fence_after_sync();
                 float sv[8];
-                const uint32_t sb = tmem + lane_base + s_col<kNSq, kNSo>(c & 1);
+                const uint32_t sb = tmem + lane_base + s_col<kNSq, kNSo>(cc & 1);
                 float scl[kGT];
                 if constexpr (kE4m3) {
                     ld_parts(std::integral_constant<int, kQParts>{}, sb, sv);
 #pragma unroll
                     for (int j = 0; j < kGT; ++j) scl[j] = qscale[c0 + j];
                 } else {
-                    tc::tmem_ld<8>(sb + c0, sv);
+                    tc::tmem_ld<kGT>(sb + hg + c0, sv);
 #pragma unroll
                     for (int j = 0; j < kGT; ++j) scl[j] = p.scale_log2;
                 }
@@ -598,15 +669,15 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
             // Lazy running max: a CTA-wide flag says whether any logit of the
             // chunk beats its head's running max by more than 2^8; only then
             // are the per-head chunk maxima reduced and the state rescaled.
-            if (__any_sync(0xffffffffu, exceed) && lane == 0) lazy_flag[c & 3] = 1;
+            if (__any_sync(0xffffffffu, exceed) && lane == 0) lazy_flag[cc & 3] = 1;
             softmax_sync<kST>();
-            const bool update = lazy_flag[c & 3] != 0;
-            if (tid == 0) lazy_flag[(c + 2) & 3] = 0;  // slot of chunk c + 2: its readers are done
+            const bool update = lazy_flag[cc & 3] != 0;
+            if (tid == 0) lazy_flag[(cc + 2) & 3] = 0;  // slot of chunk cc + 2: its readers are done
             float alpha[kGT];
 #pragma unroll
             for (int j = 0; j < kGT; ++j) alpha[j] = 1.f;
             if (update) {  // uniform across the softmax threads
-                float *rc = red + (c & 1) * 4 * kN;  // [quadrant][column]
+                float *rc = red + (cc & 1) * 4 * kN;  // [quadrant][column]
 #pragma unroll
                 for (int j = 0; j < kGT; ++j) {
                     float v = x[j];
@@ -640,9 +711,9 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                     float wa = 0.f, wb = 0.f, f = 1.f;
 #pragma unroll
                     for (int k = 0; k < kPParts; ++k) {
-                        const uint16_t cc = float2_to_e4m3x2(a, b);
-                        const float2 d = e4m3x2_to_float2(cc);
-                        pc[k][j / 2] = cc;
+                        const uint16_t code = float2_to_e4m3x2(a, b);
+                        const float2 d = e4m3x2_to_float2(code);
+                        pc[k][j / 2] = code;
                         wa = fmaf(d.x, f, wa);
                         wb = fmaf(d.y, f, wb);
                         a = (a - d.x) * 16.f;
@@ -660,16 +731,14 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                     l[j] += E::to_float(pv[j]);  // the rounded weight the MMA sees
                 }
             }
-            if (cl > 0) epilogue(c - 1);  // MMA2(c-1) done: the P tile is free again
-#pragma unroll
-            for (int j = 0; j < kGT; ++j) alpha_prev[j] = alpha[j];
+            const bool o_prev = cl > 0 && wait_o(cc - 1);
             if (c == nch - 1 && has_tail && ok && c0 == 0) {
                 // Rows of the partial last block past the context come from the
                 // pool and may hold anything (NaN): zero them in the V tile
                 // once it has landed, so 0 * V stays 0 in the PV product.
-                const int st = c % kStages;
+                const int st = cc % kStages;
                 unsigned char *vt = v_t + st * kStageBytes;
-                if (wait_ok(&v_full[st], (c / kStages) & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
+                if (wait_ok(&v_full[st], (cc / kStages) & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
 #pragma unroll
                     for (int j = 0; j < (kE4m3 ? 1 : 2); ++j)  // E4M3: a token's codes are one 128-byte row
 #pragma unroll
@@ -687,21 +756,28 @@ __global__ void __launch_bounds__(tc_threads(G), tc_ctas_per_sm(G))
                         p_t[tc::sw128_offset8(k * G + c0 + j, t)] = (unsigned char)(pc[k][j / 2] >> (8 * (j & 1)));
             } else {
                 // two 64-token regions; this thread writes rows c0 .. c0 +
-                // (16 / (kSW / 4)) - 1 (its columns, then zero rows up to 16)
+                // (16 / (kSW / 4)) - 1: its columns of the chunk's head (rows
+                // hg .. hg + kGT - 1), zeros in the other rows
                 unsigned char *pr = p_t + (t >> 6) * (kN * 128);
                 constexpr int kRowsW = kN / (kSW / 4);
 #pragma unroll
                 for (int j = 0; j < kRowsW; ++j) {
-                    const T v = j < kGT ? pv[j < kGT ? j : 0] : E::from_float(0.f);
+                    T v = E::from_float(0.f);
+#pragma unroll
+                    for (int jj = 0; jj < kGT; ++jj)
+                        if (j == hg + jj) v = pv[jj];
                     *reinterpret_cast<T *>(pr + tc::sw128_offset(c0 + j, t & 63)) = v;
                 }
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
             mbar_arrive(p_full);
+            if (o_prev) load_o(cc - 1, hg);
+#pragma unroll
+            for (int j = 0; j < kGT; ++j) alpha_prev[j] = alpha[j];
         }
-        epilogue(nch - 1);
-        finalize((nch - 1) / cpp);
+        epilogue(nct - 1, hh * G);
+        finalize(hh, (nch - 1) / cpp);
     }
 
     tc::fence_before_sync();
@@ -760,7 +836,7 @@ bool encode_cache_map(CUtensorMap *map, const void *base, int64_t rows, bool bf1
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int G, bool kMasked, bool kFp8 = false>
+template <typename T, int G, bool kMasked, bool kFp8 = false, int kHpc = 1>
 cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     const int64_t rows = p.num_blocks * p.num_kv_heads * kBlock;
     CUtensorMap tk, tv;
@@ -768,15 +844,16 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
                          : encode_cache_map(&tk, p.k_cache, rows, std::is_same<T, __nv_bfloat16>::value) &&
                                encode_cache_map(&tv, p.v_cache, rows, std::is_same<T, __nv_bfloat16>::value);
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = decode_tc_kernel<T, G, kMasked, kFp8>;
+    auto kern = decode_tc_kernel<T, G, kMasked, kFp8, kHpc>;
     static FuncAttrCache attrs;
     constexpr int kSmem = TcLayout(G, kFp8).bytes;
-    static_assert(kSmem * tc_ctas_per_sm(G) + 1024 * tc_ctas_per_sm(G) <= 228 * 1024,
+    static_assert(kSmem * tc_ctas_per_sm(G, kFp8) + 1024 * tc_ctas_per_sm(G, kFp8) <= 228 * 1024,
                   "the CTAs per SM must fit in shared memory");
     cudaError_t e = ensure_smem(kern, kSmem, attrs, /*max_carveout=*/true);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3((p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, p.num_kv_heads, p.num_seqs),
-                   dim3(tc_threads(G)), kSmem, stream, p, tk, tv,
+    if (p.heads_per_cta != kHpc || p.num_kv_heads % kHpc != 0) return cudaErrorInvalidValue;
+    e = launch_pdl(kern, dim3((p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, p.num_kv_heads / kHpc, p.num_seqs),
+                   dim3(tc_threads(G, kFp8)), kSmem, stream, p, tk, tv,
                    (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
@@ -784,6 +861,15 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
 
 template <typename T, bool kMasked>
 cudaError_t launch_tc_m(const DecodeParams &p, int rows, cudaStream_t stream) {
+    if constexpr (!kMasked) {
+        if (p.heads_per_cta == 2) {  // two KV heads per CTA (plain decode, groups of 4 or 8)
+            switch (rows) {
+                case 4: return launch_tc_t<T, 4, false, false, 2>(p, stream);
+                case 8: return launch_tc_t<T, 8, false, false, 2>(p, stream);
+                default: return cudaErrorInvalidValue;
+            }
+        }
+    }
     switch (rows) {
         case 4: return launch_tc_t<T, 4, kMasked>(p, stream);
         case 8: return launch_tc_t<T, 8, kMasked>(p, stream);

@@ -127,11 +127,23 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// The first N (8 or 16) columns of this thread's TMEM lane.
+// 4 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float *v) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// The first N (4, 8 or 16) columns of this thread's TMEM lane.
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, float *v) {
-    static_assert(N == 8 || N == 16, "8 or 16 columns");
-    if constexpr (N == 8) tmem_ld8(taddr, v);
+    static_assert(N == 4 || N == 8 || N == 16, "4, 8 or 16 columns");
+    if constexpr (N == 4) tmem_ld4(taddr, v);
+    else if constexpr (N == 8) tmem_ld8(taddr, v);
     else tmem_ld16(taddr, v);
 }
 

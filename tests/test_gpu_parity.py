@@ -139,6 +139,23 @@ def gpu_decode(p: Paged, scale: float, P: int = 0) -> torch.Tensor:
     return out
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("g,maxlen", [(4, 300), (8, 300), (4, 2100), (8, 2100)])
+def test_two_kv_heads_per_cta(orc, dtype, g, maxlen):
+    """A batch of 240 sequences (8 KV heads, groups of 4 or 8, plain decode)
+    makes the library stream two KV heads per tensor-core CTA, the query rows
+    of both heads sharing the Q tile: short contexts in one partition, and
+    contexts up to 2100 tokens split into 1024-token partitions and merged.
+    Every row against the oracle, lengths 1, 16, 17, 128, 129 and ragged."""
+    rng = np.random.default_rng(700 + g + maxlen + (dtype == "bf16"))
+    S, Hk, D = 240, 8, 128
+    lens = rng.integers(1, maxlen + 1, size=S)
+    lens[:6] = [1, 16, 17, 128, 129, maxlen]
+    p = Paged(rng, lens, Hk * g, Hk, D, dtype)
+    scale = float(np.float32(1 / np.sqrt(D)))
+    compare(gpu_decode(p, scale), p.run(orc, scale), dtype, f"two heads per CTA g={g} maxlen={maxlen}")
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
