@@ -109,7 +109,7 @@ int sm_count() {
 // own partial and the merge is unchanged.
 int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows, bool fp8) {
     if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= 64) return 1;
-    const int64_t slots = (int64_t)sm_count() * (rows > 8 || fp8 ? 2 : 3);  // resident CTAs per SM
+    const int64_t slots = (int64_t)sm_count() * (rows > 8 || (fp8 && rows >= 8) ? 2 : 3);  // resident CTAs per SM
     const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
     int ppc = 64 / pl.part_blocks;
     while (ppc > 1 && pairs * ((pl.max_parts + ppc - 1) / ppc) < 2 * slots) ppc >>= 1;

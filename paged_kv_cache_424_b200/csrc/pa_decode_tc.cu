@@ -80,12 +80,22 @@ __device__ __forceinline__ uint32_t o_col(int b) { return (uint32_t)((2 + b) * t
 static_assert(tc_tmem_cols(16, 16) == 64 && tc_tmem_cols(32, 32) == 128 && tc_tmem_cols(48, 64) == 256,
               "TMEM columns per CTA");
 
+// FP8 caches with 8 or 16 query rows per KV head take the "wide" shape: 8
+// softmax warps (two per TMEM lane quadrant, each thread holding half the
+// columns: the E4M3 weight split is the per-chunk work that sets the pace
+// there) at 2 CTAs per SM, with three stages per operand.  With 4 rows the
+// 3-CTA shape wins (measured: gqa8b over FP8 152 us against 188 us wide,
+// long70b over FP8 175 us against 164 us wide): a batch of short
+// sequences needs the third CTA per SM to cover each CTA's start.
+__host__ __device__ constexpr bool tc_wide(int G, bool e4m3) { return G > 8 || (e4m3 && G >= 8); }
+
 // K / V stages: a 16-bit chunk fills a 32 KiB tile area (two 64-dim
-// regions), one stage per operand at 3 CTAs per SM; E4M3 codes take 16 KiB
-// a chunk, three stages per operand at 2 CTAs per SM, so the loads of the
-// next chunks overlap the products and the softmax of the current one.
+// regions), one stage per operand; E4M3 codes take 16 KiB a chunk, two
+// stages per operand at 3 CTAs per SM, three with the wide FP8 shape, so
+// the loads of the next chunks overlap the products and the softmax of the
+// current one.
 constexpr int kMaxStages = 3;
-__host__ __device__ constexpr int tc_stages(bool e4m3) { return e4m3 ? 3 : 1; }
+__host__ __device__ constexpr int tc_stages(int G, bool e4m3) { return !e4m3 ? 1 : tc_wide(G, e4m3) ? 3 : 2; }
 __host__ __device__ constexpr int tc_stage_bytes(bool e4m3) { return e4m3 ? kRegion : 2 * kRegion; }
 
 // Shared-memory layout (bytes from the 1024-aligned base): K tile area,
@@ -98,7 +108,8 @@ constexpr int kNumBars = 4 * kMaxStages + 6;
 struct TcLayout {
     int k_off, v_off, q_off, p_off, red_off, bar_off, misc_off, qscale_off, bytes;
     __host__ __device__ constexpr TcLayout(int G, bool e4m3)
-        : k_off(0), v_off(tc_stages(e4m3) * tc_stage_bytes(e4m3)), q_off(2 * tc_stages(e4m3) * tc_stage_bytes(e4m3)),
+        : k_off(0), v_off(tc_stages(G, e4m3) * tc_stage_bytes(e4m3)),
+          q_off(2 * tc_stages(G, e4m3) * tc_stage_bytes(e4m3)),
           p_off(q_off + (e4m3 ? tc_cols_s(G, true) * 128 : 2 * kN * 128)),
           red_off(p_off + (e4m3 ? tc_cols_o(G, true) * 128 : 2 * kN * 128)), bar_off(red_off + 2 * 4 * kN * 4),
           misc_off(bar_off + kNumBars * 8), qscale_off(misc_off + 32),
@@ -199,15 +210,12 @@ __device__ __forceinline__ void produce_tile(const DecodeParams &p, const CUtens
 // anyway (80 per thread for 3 CTAs of 7 or 8 warps per SM); with the fourth
 // warp present it spills far less in the softmax loop (measured with
 // -Xptxas -v: 44 -> 4 bytes for 8 columns).
-// FP8 caches: 8 softmax warps whatever the group, two per quadrant, each
-// thread holding half the columns (the E4M3 weight split is the per-chunk
-// work that sets the pace there).
-__host__ __device__ constexpr int tc_soft_warps(int G, bool e4m3) { return G > 8 || e4m3 ? 8 : 4; }
+__host__ __device__ constexpr int tc_soft_warps(int G, bool e4m3) { return tc_wide(G, e4m3) ? 8 : 4; }
 __host__ __device__ constexpr int tc_threads(int G, bool e4m3) { return (tc_soft_warps(G, e4m3) + 4) * 32; }
 
 // CTAs per SM: 3 (registers and shared memory both allow it) except with 16
 // columns, whose 11 warps fit twice.
-__host__ __device__ constexpr int tc_ctas_per_sm(int G, bool e4m3) { return G > 8 || e4m3 ? 2 : 3; }
+__host__ __device__ constexpr int tc_ctas_per_sm(int G, bool e4m3) { return tc_wide(G, e4m3) ? 2 : 3; }
 
 // G: columns of S (query rows per KV head: the group, or group x query
 // tokens with kMasked, padded to a power of two).
@@ -230,13 +238,13 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int kSW = tc_soft_warps(G, kFp8);  // softmax warps
     constexpr int kST = kSW * 32;                // softmax threads
-    constexpr int kGT = kFp8 ? G / 2 : G > 8 ? 8 : G;  // columns per softmax thread
+    constexpr int kGT = tc_soft_warps(G, kFp8) == 8 ? G / 2 : G;  // columns per softmax thread
     constexpr int kWarpK = kSW, kWarpMma = kSW + 1, kWarpV = kSW + 2;
     constexpr bool kE4m3 = kFp8;                 // both products on the E4M3 codes
     constexpr int kNSq = tc_cols_s(G, kE4m3);    // columns of S
     constexpr int kNSo = tc_cols_o(G, kE4m3);    // columns of O
     constexpr uint32_t kTmemCols = tc_tmem_cols(kNSq, kNSo);
-    constexpr int kStages = tc_stages(kE4m3);
+    constexpr int kStages = tc_stages(G, kE4m3);
     constexpr int kStageBytes = tc_stage_bytes(kE4m3);
     constexpr TcLayout Lay(G, kE4m3);
     extern __shared__ __align__(1024) unsigned char smem[];
