@@ -33,7 +33,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Q tile) then amortises over more chunks while long contexts still give
 // thousands of CTAs.  The merge costs ~1-2% of the KV traffic either way.
 constexpr int kAutoPartitionSimt = 512;
-constexpr int kAutoPartitionTc = 1024;
+constexpr int kAutoPartitionTc = 1024;  // 2048 for large batches (tc_auto_partition)
 constexpr int kMaxPartitionTokens = 32768;
 
 bool kv_fp8(const pa_dims *d) { return d->kv_dtype == PA_FP8_E4M3; }
@@ -100,18 +100,28 @@ int sm_count() {
     return 148;
 }
 
+// Resident tensor-core CTAs on the device: 2 per SM with 16 rows or the
+// wide FP8 shape, 3 otherwise.
+int64_t tc_slots(int rows, bool fp8) { return (int64_t)sm_count() * (rows > 8 || (fp8 && rows >= 8) ? 2 : 3); }
+
+// Tokens one tensor-core CTA streams at most when it groups partitions:
+// 1024 over 16-bit caches, 2048 over FP8 ones, whose chunks take half the
+// time and so pay relatively twice the per-CTA cost.
+int tc_group_blocks(bool fp8) { return fp8 ? 128 : 64; }
+
 // Partitions one tensor-core CTA streams back to back: partitions shorter
-// than 1024 tokens (8 chunks) that start on a chunk are grouped up to 1024
-// tokens per CTA, which saves the per-CTA set-up (TMEM, barriers, Q tile,
-// pipeline fill; measured: the 70B shape at 512-token partitions ran at
-// 0.78 of the copy roofline against 0.87 at 1024), as long as the grid
-// keeps at least two waves of resident CTAs.  Each partition still gets its
-// own partial and the merge is unchanged.
+// than the group size that start on a chunk are grouped up to it per CTA,
+// which saves the per-CTA set-up (TMEM, barriers, Q tile, pipeline fill and
+// drain; measured: the 70B shape at 512-token partitions ran at 0.78 of the
+// copy roofline against 0.87 at 1024), as long as the grid keeps at least
+// two waves of resident CTAs.  Each partition still gets its own partial and
+// the merge is unchanged.
 int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows, bool fp8) {
-    if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= 64) return 1;
-    const int64_t slots = (int64_t)sm_count() * (rows > 8 || (fp8 && rows >= 8) ? 2 : 3);  // resident CTAs per SM
+    const int group = tc_group_blocks(fp8);
+    if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= group) return 1;
+    const int64_t slots = tc_slots(rows, fp8);
     const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
-    int ppc = 64 / pl.part_blocks;
+    int ppc = group / pl.part_blocks;
     while (ppc > 1 && pairs * ((pl.max_parts + ppc - 1) / ppc) < 2 * slots) ppc >>= 1;
     return ppc;
 }
@@ -132,6 +142,16 @@ int tc_heads_per_cta(const Plan &pl, const pa_dims *d, int rows, bool plain) {
     return hpc;
 }
 
+// Automatic partition of the tensor-core kernel: 2048 tokens when the batch
+// still gives two waves of resident CTAs at that size (a CTA then pays its
+// set-up, first loads and drain once per up to 16 chunks; measured on the
+// 8B continuous-batching step: 156 us against 159 us at 1024 over a 16-bit
+// cache, 118 us against 141 us over an FP8 one), else 1024.
+int tc_auto_partition(const pa_dims *d, int ctx_blocks, int rows, bool fp8) {
+    const int64_t ctas = (int64_t)d->num_seqs * d->num_kv_heads * ((ctx_blocks + 127) / 128);
+    return ctas >= 2 * tc_slots(rows, fp8) ? 2 * kAutoPartitionTc : kAutoPartitionTc;
+}
+
 pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
                     int32_t q_len = 1, int32_t window = 0) {
     if (max_context_len < 0) return fail(PA_ERR_SHAPE, "max_context_len %d < 0", max_context_len);
@@ -142,8 +162,7 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         return fail(PA_ERR_SHAPE, "partition_tokens %d must be 0 or a positive multiple of 16 up to %d",
                     partition_tokens, kMaxPartitionTokens);
     const int g = d->num_heads / d->num_kv_heads;
-    const bool tc = tc_rows(d, row_capacity(g * q_len)) != 0;
-    const int P = partition_tokens != 0 ? partition_tokens : tc ? kAutoPartitionTc : kAutoPartitionSimt;
+    const int rows = tc_rows(d, row_capacity(g * q_len));
     int ctx_blocks = (max_context_len + 15) / 16;
     if (window > 0) {
         // attended positions of a sequence span at most window + q_len - 1
@@ -151,6 +170,9 @@ pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition
         const int64_t span_blocks = ((int64_t)window + q_len - 1 + 15) / 16 + 1;
         if (span_blocks < ctx_blocks) ctx_blocks = (int)span_blocks;
     }
+    const int P = partition_tokens != 0 ? partition_tokens
+                  : rows                ? tc_auto_partition(d, ctx_blocks, rows, kv_fp8(d))
+                                        : kAutoPartitionSimt;
     int part_blocks = P / 16;
     const int max_parts = ctx_blocks == 0 ? 1 : (ctx_blocks + part_blocks - 1) / part_blocks;
     if (max_parts == 1) part_blocks = ctx_blocks > 0 ? ctx_blocks : 1;  // one partition: size it to the context

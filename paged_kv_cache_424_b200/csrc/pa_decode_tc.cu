@@ -29,7 +29,9 @@
 //           other chunks), writes P (same 16-bit type as V) into a swizzled
 //           tile, and accumulates O chunk by chunk in registers.
 // Shared memory: K tile 32 KiB + V tile 32 KiB + Q 4 KiB + P 4 KiB (+ <1 KiB)
-// = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.
+// = 74 KiB, three CTAs per SM; TMEM: 64 columns per CTA.  With 16 columns
+// (two CTAs per SM) a second V stage (+32 KiB) lets the V load of the next
+// chunk overlap the current chunk's softmax and PV product.
 // FP8 E4M3 caches: a chunk's codes take 16 KiB (128-byte swizzle), so each
 // 32 KiB tile area holds two stages and the loads of chunk c + 1 overlap the
 // products of chunk c.  Both products run E4M3 x E4M3 on the codes as
@@ -96,6 +98,10 @@ __host__ __device__ constexpr bool tc_wide(int G, bool e4m3) { return G > 8 || (
 // current one.
 constexpr int kMaxStages = 3;
 __host__ __device__ constexpr int tc_stages(int G, bool e4m3) { return !e4m3 ? 1 : tc_wide(G, e4m3) ? 3 : 2; }
+// V stages: a second one for 16-bit caches with 16 columns, whose two CTAs
+// per SM leave room for it; the V load of chunk c + 1 then overlaps the
+// softmax and the PV product of chunk c instead of starting after them.
+__host__ __device__ constexpr int tc_stages_v(int G, bool e4m3) { return !e4m3 && G > 8 ? 2 : tc_stages(G, e4m3); }
 __host__ __device__ constexpr int tc_stage_bytes(bool e4m3) { return e4m3 ? kRegion : 2 * kRegion; }
 
 // Shared-memory layout (bytes from the 1024-aligned base): K tile area,
@@ -109,7 +115,7 @@ struct TcLayout {
     int k_off, v_off, q_off, p_off, red_off, bar_off, misc_off, qscale_off, bytes;
     __host__ __device__ constexpr TcLayout(int G, bool e4m3)
         : k_off(0), v_off(tc_stages(G, e4m3) * tc_stage_bytes(e4m3)),
-          q_off(2 * tc_stages(G, e4m3) * tc_stage_bytes(e4m3)),
+          q_off((tc_stages(G, e4m3) + tc_stages_v(G, e4m3)) * tc_stage_bytes(e4m3)),
           p_off(q_off + (e4m3 ? tc_cols_s(G, true) * 128 : 2 * kN * 128)),
           red_off(p_off + (e4m3 ? tc_cols_o(G, true) * 128 : 2 * kN * 128)), bar_off(red_off + 2 * 4 * kN * 4),
           misc_off(bar_off + kNumBars * 8), qscale_off(misc_off + 32),
@@ -124,6 +130,14 @@ __device__ __forceinline__ bool wait_ok(uint64_t *bar, uint32_t parity, int *fai
     if (mbar_wait(bar, parity)) return true;
     atomicOr(fail, 1);
     return false;
+}
+
+// Maximum of v over the warp (NaN inputs ignored, like fmaxf), one
+// instruction on sm_100a.
+__device__ __forceinline__ float warp_max(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 // Named barrier 1 over the N softmax threads.
@@ -244,7 +258,8 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     constexpr int kNSq = tc_cols_s(G, kE4m3);    // columns of S
     constexpr int kNSo = tc_cols_o(G, kE4m3);    // columns of O
     constexpr uint32_t kTmemCols = tc_tmem_cols(kNSq, kNSo);
-    constexpr int kStages = tc_stages(G, kE4m3);
+    constexpr int kStages = tc_stages(G, kE4m3);      // K stages
+    constexpr int kStagesV = tc_stages_v(G, kE4m3);   // V stages
     constexpr int kStageBytes = tc_stage_bytes(kE4m3);
     constexpr TcLayout Lay(G, kE4m3);
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -331,6 +346,8 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < kStagesV; ++i) {
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
         }
@@ -351,7 +368,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
         produce_tile<kE4m3, kStages, kHpc>(p, &tmap_k, k_t, k_full, k_empty, fail, s, kvh, b0, nb, nch, oob_row,
                                            lane, pre);
     } else if (warp == kWarpV) {
-        produce_tile<kE4m3, kStages, kHpc>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row,
+        produce_tile<kE4m3, kStagesV, kHpc>(p, &tmap_v, v_t, v_full, v_empty, fail, s, kvh, b0, nb, nch, oob_row,
                                            lane, pre);
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer ------------------------------
@@ -363,7 +380,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
             const uint32_t kb = smem_addr(k_t), vb = smem_addr(v_t), qb = smem_addr(q_t), pb = smem_addr(p_t);
             // PV(c): O^T = V^T . P^T into O buffer c & 1
             auto issue_pv = [&](int c) {
-                const int st = c % kStages;
+                const int st = c % kStagesV;
                 tc::fence_after_sync();
                 const uint32_t vs = vb + st * kStageBytes;
                 if constexpr (kE4m3) {
@@ -427,7 +444,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                     progress = true;
                 }
                 if (npv < ns && mbar_test(p_full, npv & 1) &&
-                    mbar_test(&v_full[npv % kStages], (npv / kStages) & 1)) {
+                    mbar_test(&v_full[npv % kStagesV], (npv / kStagesV) & 1)) {
                     issue_pv(npv);
                     ++npv;
                     progress = true;
@@ -688,9 +705,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                 float *rc = red + (cc & 1) * 4 * kN;  // [quadrant][column]
 #pragma unroll
                 for (int j = 0; j < kGT; ++j) {
-                    float v = x[j];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    const float v = warp_max(x[j]);
                     if (lane == 0) rc[(kSW == 8 ? warp & 3 : warp) * kN + c0 + j] = v;
                 }
                 softmax_sync<kST>();
@@ -744,9 +759,9 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                 // Rows of the partial last block past the context come from the
                 // pool and may hold anything (NaN): zero them in the V tile
                 // once it has landed, so 0 * V stays 0 in the PV product.
-                const int st = cc % kStages;
+                const int st = cc % kStagesV;
                 unsigned char *vt = v_t + st * kStageBytes;
-                if (wait_ok(&v_full[st], (cc / kStages) & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
+                if (wait_ok(&v_full[st], (cc / kStagesV) & 1, fail) && tok >= L && tok < (b0 + nb) * kBlock) {
 #pragma unroll
                     for (int j = 0; j < (kE4m3 ? 1 : 2); ++j)  // E4M3: a token's codes are one 128-byte row
 #pragma unroll

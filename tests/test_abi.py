@@ -72,6 +72,14 @@ def test_workspace_plan(lib):
     assert lib.pa_decode_num_partitions(d, 4096, 4096) == 1
     assert lib.pa_decode_workspace_size(d, 4096, 4096) == 0
     assert lib.pa_decode_num_partitions(d, 0, 0) == 1
+    # a batch that fills two waves of resident CTAs at 2048-token partitions
+    # takes them (148 SMs x 3 CTAs when no device answers)
+    big = _dims(lib, num_seqs=256)
+    assert lib.pa_decode_num_partitions(big, 4096, 0) == 2
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, max_blocks_per_seq=512), 4097, 0) == 3
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=lib.PA_FP8_E4M3), 4096, 0) == 2
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=16), 4096, 0) == 4  # 256 CTAs at 2048: 1024
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, num_heads=8), 4096, 0) == 8  # CUDA-core: 512
 
 
 @pytest.mark.parametrize("kw,status", [
