@@ -33,7 +33,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Q tile) then amortises over more chunks while long contexts still give
 // thousands of CTAs.  The merge costs ~1-2% of the KV traffic either way.
 constexpr int kAutoPartitionSimt = 512;
-constexpr int kAutoPartitionTc = 1024;  // 2048 for large batches (tc_auto_partition)
+constexpr int kAutoPartitionTc = 1024;  // up to 4x for large batches (tc_auto_partition)
 constexpr int kMaxPartitionTokens = 32768;
 
 bool kv_fp8(const pa_dims *d) { return d->kv_dtype == PA_FP8_E4M3; }
@@ -142,14 +142,20 @@ int tc_heads_per_cta(const Plan &pl, const pa_dims *d, int rows, bool plain) {
     return hpc;
 }
 
-// Automatic partition of the tensor-core kernel: 2048 tokens when the batch
-// still gives two waves of resident CTAs at that size (a CTA then pays its
-// set-up, first loads and drain once per up to 16 chunks; measured on the
-// 8B continuous-batching step: 156 us against 159 us at 1024 over a 16-bit
-// cache, 118 us against 141 us over an FP8 one), else 1024.
+// Automatic partition of the tensor-core kernel: the largest of 4096 (FP8
+// caches only), 2048 and 1024 tokens at which the batch still gives two
+// waves of resident CTAs.  A CTA pays its set-up, first loads and drain
+// once per partition, and over an FP8 cache its chunks take half the time
+// (measured on the 8B continuous-batching step: 156 us at 2048 against 159
+// at 1024 over a 16-bit cache; 102 us at 4096, 109 at 2048 and 141 at 1024
+// over an FP8 one).
 int tc_auto_partition(const pa_dims *d, int ctx_blocks, int rows, bool fp8) {
-    const int64_t ctas = (int64_t)d->num_seqs * d->num_kv_heads * ((ctx_blocks + 127) / 128);
-    return ctas >= 2 * tc_slots(rows, fp8) ? 2 * kAutoPartitionTc : kAutoPartitionTc;
+    const int64_t pairs = (int64_t)d->num_seqs * d->num_kv_heads;
+    for (int P = fp8 ? 4 * kAutoPartitionTc : 2 * kAutoPartitionTc; P > kAutoPartitionTc; P /= 2) {
+        const int blocks = P / 16;
+        if (pairs * ((ctx_blocks + blocks - 1) / blocks) >= 2 * tc_slots(rows, fp8)) return P;
+    }
+    return kAutoPartitionTc;
 }
 
 pa_status make_plan(const pa_dims *d, int32_t max_context_len, int32_t partition_tokens, Plan *pl,
@@ -241,6 +247,14 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     // the plain tensor-core variant: one query token, no window, unscaled 16-bit V
     const bool plain = tc && !fp8 && q_len == 1 && window == 0 && v_scale == 1.f;
     p.heads_per_cta = plain && p.parts_per_cta == 1 ? tc_heads_per_cta(pl, dims, tc, true) : 1;
+    // Over an FP8 cache the tensor-core grid launches every sequence's first
+    // partition before any later one: the CTAs of partitions past short
+    // sequences (which read the context length and leave) then come in the
+    // second half of the launch instead of between the busy ones (measured
+    // on the 8B continuous-batching step: 116.7 -> 107.5 us; the 16-bit
+    // shapes lost 1-2 % with it and keep the sequence-major order).
+    const int64_t part_groups = (pl.max_parts + p.parts_per_cta - 1) / p.parts_per_cta;
+    p.part_major = tc && fp8 && part_groups <= 65535 ? 1 : 0;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e = tc ? pa::launch_decode_tc(p, dims->dtype, tc, fp8, cs)
                        : pa::launch_decode_partitioned(p, dims->dtype, dims->head_dim, rows, fp8, cs);

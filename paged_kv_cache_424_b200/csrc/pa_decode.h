@@ -36,6 +36,7 @@ struct DecodeParams {
     const int32_t *seq_order;    // nullptr, or the sequence each blockIdx.z visits
     int32_t parts_per_cta;       // tensor-core kernel: consecutive partitions one CTA streams (1 elsewhere)
     int32_t heads_per_cta;       // tensor-core kernel, plain decode: consecutive KV heads one CTA streams (1 elsewhere)
+    int32_t part_major;          // tensor-core kernel: grid (head, position, partition) instead of (partition, head, position)
 };
 
 // Whether a launch needs per-row position masks (several query tokens or a

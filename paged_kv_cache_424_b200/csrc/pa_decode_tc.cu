@@ -122,6 +122,35 @@ struct TcLayout {
           bytes(qscale_off + kN * 4) {}
 };
 
+// Two fp32 values packed in one 64-bit register pair, and the sm_100
+// packed arithmetic on them: each lane is the ordinary IEEE round-to-nearest
+// single-precision operation, two per instruction.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 __device__ __forceinline__ bool is_failed(const int *f) { return *reinterpret_cast<const volatile int *>(f) != 0; }
 
 // Bounded wait that gives up at once when another thread already failed.
@@ -282,15 +311,23 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     // each, partitions part0 .. part0 + ppc - 1 (those that exist), back to
     // back: one set-up, one pipeline, one partial per (head, partition)
     constexpr int hpc = kHpc;
-    const int kvh = blockIdx.y * hpc;
+    // Grid: x = partition group, y = KV head group, z = schedule position (a
+    // sequence's CTAs launch together), or with p.part_major x = KV head
+    // group, y = schedule position, z = partition group (every sequence's
+    // first partition launches before any later one)
+    const bool pm = p.part_major != 0;
+    const int g_part = pm ? (int)blockIdx.z : (int)blockIdx.x;
+    const int g_head = pm ? (int)blockIdx.x : (int)blockIdx.y;
+    const int g_seq = pm ? (int)blockIdx.y : (int)blockIdx.z;
+    const int kvh = g_head * hpc;
     const int ppc = p.parts_per_cta;
-    const int part0 = blockIdx.x * ppc;
+    const int part0 = g_part * ppc;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.num_heads, head0 = kvh * G;  // head0: unmasked launches (group == G, q_len == 1)
     T *out = reinterpret_cast<T *>(p.out);
     pdl_launch_dependents();
     pdl_wait();
-    const int s = scheduled_seq(p, blockIdx.z, part0 == 0 && blockIdx.y == 0 && tid == 0);
+    const int s = scheduled_seq(p, g_seq, part0 == 0 && g_head == 0 && tid == 0);
     if (s < 0) return;
     // Without a window a CTA's slice of the table starts at part0 *
     // part_blocks whatever the context length: the producers issue its first
@@ -311,7 +348,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     };
     const int rows = kMasked ? p.group * p.q_len : G * hpc;  // real Q rows of the CTA
 
-    const SeqSplit sp = seq_split(p, s, part0 == 0 && blockIdx.y == 0 && tid == 0);
+    const SeqSplit sp = seq_split(p, s, part0 == 0 && g_head == 0 && tid == 0);
     const int L = sp.L, nblk = sp.nblk, nparts = sp.nparts;
     if (part0 >= nparts) return;
     const int nmine = min(ppc, nparts - part0);  // partitions of this CTA
@@ -539,23 +576,35 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
         // TMEM column k G + c0 + j divided by 16^k (Horner from the last part)
         auto ld_parts = [&](auto np, uint32_t taddr, float *v) {
             constexpr int NP = decltype(np)::value;
+            const uint64_t sixteenth = pk2(0.0625f, 0.0625f);
             if constexpr (G == 4) {
                 float t16[16];
                 tc::tmem_ld<16>(taddr, t16);
 #pragma unroll
-                for (int j = 0; j < kGT; ++j) {
-                    float a = t16[(NP - 1) * 4 + c0 + j];
+                for (int j = 0; j < kGT; j += 2) {
+                    uint64_t a = pk2(t16[(NP - 1) * 4 + c0 + j], t16[(NP - 1) * 4 + c0 + j + 1]);
 #pragma unroll
-                    for (int k = NP - 2; k >= 0; --k) a = fmaf(a, 0.0625f, t16[k * 4 + c0 + j]);
-                    v[j] = a;
+                    for (int k = NP - 2; k >= 0; --k)
+                        a = fma2(a, sixteenth, pk2(t16[k * 4 + c0 + j], t16[k * 4 + c0 + j + 1]));
+                    const float2 r = up2(a);
+                    v[j] = r.x;
+                    v[j + 1] = r.y;
                 }
             } else {
                 float b[kGT];
+                uint64_t a[kGT / 2];
 #pragma unroll
                 for (int k = NP - 1; k >= 0; --k) {
                     tc::tmem_ld<kGT>(taddr + G * k + c0, b);
 #pragma unroll
-                    for (int j = 0; j < kGT; ++j) v[j] = k == NP - 1 ? b[j] : fmaf(v[j], 0.0625f, b[j]);
+                    for (int j = 0; j < kGT; j += 2)
+                        a[j / 2] = k == NP - 1 ? pk2(b[j], b[j + 1]) : fma2(a[j / 2], sixteenth, pk2(b[j], b[j + 1]));
+                }
+#pragma unroll
+                for (int j = 0; j < kGT; j += 2) {
+                    const float2 r = up2(a[j / 2]);
+                    v[j] = r.x;
+                    v[j + 1] = r.y;
                 }
             }
         };
@@ -729,22 +778,25 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
 #pragma unroll
                 for (int j = 0; j < kGT; j += 2) {
                     // a masked column may still have m = -inf: weight 0, not 2^(-inf + inf)
-                    float a = x[j] == -INFINITY ? 0.f : ex2(x[j] - m[j]);
-                    float b = x[j + 1] == -INFINITY ? 0.f : ex2(x[j + 1] - m[j + 1]);
-                    float wa = 0.f, wb = 0.f, f = 1.f;
+                    const float a = x[j] == -INFINITY ? 0.f : ex2(x[j] - m[j]);
+                    const float b = x[j + 1] == -INFINITY ? 0.f : ex2(x[j + 1] - m[j + 1]);
+                    // the pair (a, b) in one register pair: remainder r, sums w
+                    uint64_t r = pk2(a, b), w = pk2(0.f, 0.f);
+                    float f = 1.f;
 #pragma unroll
                     for (int k = 0; k < kPParts; ++k) {
-                        const uint16_t code = float2_to_e4m3x2(a, b);
+                        const float2 rf = up2(r);
+                        const uint16_t code = float2_to_e4m3x2(rf.x, rf.y);
                         const float2 d = e4m3x2_to_float2(code);
+                        const uint64_t dd = pk2(d.x, d.y);
                         pc[k][j / 2] = code;
-                        wa = fmaf(d.x, f, wa);
-                        wb = fmaf(d.y, f, wb);
-                        a = (a - d.x) * 16.f;
-                        b = (b - d.y) * 16.f;
+                        w = fma2(dd, pk2(f, f), w);
+                        r = mul2(sub2(r, dd), pk2(16.f, 16.f));  // exact: the part's rounding error, scaled
                         f *= 0.0625f;
                     }
-                    l[j] += wa;  // the weight the MMA sees (to f32 rounding)
-                    l[j + 1] += wb;
+                    const float2 wf = up2(w);
+                    l[j] += wf.x;  // the weight the MMA sees (to f32 rounding)
+                    l[j + 1] += wf.y;
                 }
             } else {
 #pragma unroll
@@ -875,9 +927,10 @@ cudaError_t launch_tc_t(const DecodeParams &p, cudaStream_t stream) {
     cudaError_t e = ensure_smem(kern, kSmem, attrs, /*max_carveout=*/true);
     if (e != cudaSuccess) return e;
     if (p.heads_per_cta != kHpc || p.num_kv_heads % kHpc != 0) return cudaErrorInvalidValue;
-    e = launch_pdl(kern, dim3((p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, p.num_kv_heads / kHpc, p.num_seqs),
-                   dim3(tc_threads(G, kFp8)), kSmem, stream, p, tk, tv,
-                   (int)rows);
+    const unsigned parts = (p.max_parts + p.parts_per_cta - 1) / p.parts_per_cta, heads = p.num_kv_heads / kHpc;
+    if (p.part_major && parts > 65535) return cudaErrorInvalidValue;
+    const dim3 grid = p.part_major ? dim3(heads, p.num_seqs, parts) : dim3(parts, heads, p.num_seqs);
+    e = launch_pdl(kern, grid, dim3(tc_threads(G, kFp8)), kSmem, stream, p, tk, tv, (int)rows);
     if (e != cudaSuccess || p.max_parts == 1) return e;
     return launch_merge_partitions(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, kD, stream);
 }

@@ -77,7 +77,11 @@ def test_workspace_plan(lib):
     big = _dims(lib, num_seqs=256)
     assert lib.pa_decode_num_partitions(big, 4096, 0) == 2
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, max_blocks_per_seq=512), 4097, 0) == 3
-    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=lib.PA_FP8_E4M3), 4096, 0) == 2
+    # over an FP8 cache up to 4096 tokens
+    f8 = lib.PA_FP8_E4M3
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=f8), 4096, 0) == 1
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=f8, max_blocks_per_seq=512), 8192, 0) == 2
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=32, kv_dtype=f8, max_blocks_per_seq=512), 8192, 0) == 4
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=16), 4096, 0) == 4  # 256 CTAs at 2048: 1024
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, num_heads=8), 4096, 0) == 8  # CUDA-core: 512
 
