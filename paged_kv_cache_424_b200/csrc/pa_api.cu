@@ -105,17 +105,17 @@ int sm_count() {
 int64_t tc_slots(int rows, bool fp8) { return (int64_t)sm_count() * (rows > 8 || (fp8 && rows >= 8) ? 2 : 3); }
 
 // Tokens one tensor-core CTA streams at most when it groups partitions:
-// 1024 over 16-bit caches, 2048 over FP8 ones, whose chunks take half the
+// 1024 over 16-bit caches, 4096 over FP8 ones, whose chunks take half the
 // time and so pay relatively twice the per-CTA cost.
-int tc_group_blocks(bool fp8) { return fp8 ? 128 : 64; }
+int tc_group_blocks(bool fp8) { return fp8 ? 256 : 64; }
 
 // Partitions one tensor-core CTA streams back to back: partitions shorter
 // than the group size that start on a chunk are grouped up to it per CTA,
 // which saves the per-CTA set-up (TMEM, barriers, Q tile, pipeline fill and
 // drain; measured: the 70B shape at 512-token partitions ran at 0.78 of the
 // copy roofline against 0.87 at 1024), as long as the grid keeps at least
-// two waves of resident CTAs.  Each partition still gets its own partial and
-// the merge is unchanged.
+// two waves of resident CTAs.  The CTA writes one partial for the group, in
+// its first partition's slot, and marks the others empty for the merge.
 int tc_parts_per_cta(const Plan &pl, int num_seqs, int num_kv_heads, int rows, bool fp8) {
     const int group = tc_group_blocks(fp8);
     if (pl.max_parts <= 1 || pl.part_blocks % 8 != 0 || pl.part_blocks >= group) return 1;

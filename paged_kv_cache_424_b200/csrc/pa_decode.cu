@@ -243,8 +243,12 @@ __device__ __forceinline__ void merge_accumulate(MergeAcc<D> &a, const float *ls
             w[k] = 0.f;
 #pragma unroll
             for (int e = 0; e < kV; ++e) v[k][e] = 0.f;
-            if (i < n) {
-                w[k] = exp2f(lse[i] - M);  // lse = -inf (no position in that partition) gives 0
+            const float li = i < n ? lse[i] : -INFINITY;
+            // lse = -inf (no position in that partition, or a partition whose
+            // tokens another partial of the same CTA holds) gives weight 0,
+            // and its o, possibly never written, is not read
+            if (li != -INFINITY) {
+                w[k] = exp2f(li - M);
                 const float *src = o_row + (int64_t)i * D + lane * kV;
                 if constexpr (kV == 4) {
                     const float4 x = *reinterpret_cast<const float4 *>(src);

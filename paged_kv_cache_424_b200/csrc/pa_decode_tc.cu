@@ -367,7 +367,11 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     const int nch = (nb + kChunkBlocks - 1) / kChunkBlocks; // chunks of 128 tokens
     // chunks per partition: partitions of several chunks start on a chunk
     // (the host sets ppc > 1 only when part_blocks is a multiple of 8)
-    const int cpp = ppc > 1 ? p.part_blocks / kChunkBlocks : nch;
+    // One partial per CTA: the partitions a CTA streams are combined into
+    // the slot of its first one, and the others are marked empty (lse =
+    // -inf, weight 0 in the merge), so the pipeline runs through partition
+    // boundaries instead of draining at each (chunks per written partial).
+    const int cpp = nch;
     const int tok0 = b0 * kBlock;
     const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
     const int nct = hpc * nch;                              // chunks of all the CTA's heads
@@ -665,7 +669,10 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                         } else {
                             const int64_t r = qr * p.max_parts + part;
                             p.ws_o[r * kD + t] = o;
-                            if (t == 0) p.ws_lse[r] = lt > 0.f ? m[j] + log2f(lt) : -INFINITY;
+                            if (t == 0) {
+                                p.ws_lse[r] = lt > 0.f ? m[j] + log2f(lt) : -INFINITY;
+                                for (int k = 1; k < nmine; ++k) p.ws_lse[r + k] = -INFINITY;
+                            }
                         }
                     } else {  // plain decode: every column has tokens, V unscaled
                         const float o = acc[j] / lt;
@@ -675,7 +682,10 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                         } else {
                             const int64_t r = qh * p.max_parts + part;
                             p.ws_o[r * kD + t] = o;
-                            if (t == 0) p.ws_lse[r] = m[j] + log2f(lt);
+                            if (t == 0) {
+                                p.ws_lse[r] = m[j] + log2f(lt);
+                                for (int k = 1; k < nmine; ++k) p.ws_lse[r + k] = -INFINITY;
+                            }
                         }
                     }
                 }

@@ -206,6 +206,20 @@ def test_long70b_reduced_fp8():
     run_and_compare(sc, partition_tokens=16)
 
 
+def test_grouped_partitions_fp8():
+    """Over an FP8 cache a CTA groups partitions up to 4096 tokens into one
+    partial: 64 sequences of up to 2048 tokens at 512-token partitions."""
+    sc = W().gqa8b(seed=72, num_seqs=64, num_steps=1, median=1500, cap=2048, num_blocks=16384)
+    run_and_compare(W().with_fp8_cache(sc), partition_tokens=512)
+
+
+def test_long70b_full_fp8_sampled():
+    """The 70B long-context batch at its stated 512-token partitions over an
+    FP8 cache (four partitions per CTA, one partial each): two sequences
+    checked against the oracle."""
+    run_and_compare(W().with_fp8_cache(W().long70b()), seqs=np.array([0, 5]))
+
+
 def test_cow_reduced_fp8():
     """Copy-on-write copies move FP8 blocks (half the bytes of a 16-bit one)."""
     sc = W().with_fp8_cache(W().cow(seed=54, num_prompts=2, num_blocks=1024))

@@ -86,6 +86,15 @@ def test_long70b_full():
     run_and_compare(W().long70b())
 
 
+def test_grouped_partitions_write_one_partial_per_cta():
+    """64 sequences of up to 2048 tokens at 512-token partitions fill two
+    waves of CTAs with two partitions per CTA: each CTA writes one partial
+    for both (in the first one's slot) and marks the other empty, and the
+    merge must give the oracle's result; lengths end anywhere in a block."""
+    sc = W().gqa8b(seed=71, num_seqs=64, num_steps=1, median=1500, cap=2048, num_blocks=16384)
+    run_and_compare(sc, partition_tokens=512)
+
+
 @pytest.mark.parametrize("every", [False, True])
 def test_cow_full(every):
     sc = W().cow(cow_every_sample=every)
