@@ -135,7 +135,8 @@ int32_t pa_decode_num_partitions(const pa_dims *dims, int32_t max_context_len,
  * max_context_len is a host-known upper bound on context_lens (it sizes the
  * partition grid); lengths above it are clamped and flagged.
  * partition_tokens: 0 = automatic (the CUDA-core kernel: 512 tokens; the
- * tensor-core kernel: the largest of 4096 (FP8 caches only), 2048 and 1024
+ * tensor-core kernel: the largest of 4096 (FP8 caches and 16 query rows
+ * per KV head only), 2048 and 1024
  * tokens at which num_seqs x num_kv_heads x ceil(max_context_len / P) still
  * reaches two waves of resident CTAs), else a positive multiple of 16; with
  * more than one

@@ -105,9 +105,11 @@ int sm_count() {
 int64_t tc_slots(int rows, bool fp8) { return (int64_t)sm_count() * (rows > 8 || (fp8 && rows >= 8) ? 2 : 3); }
 
 // Tokens one tensor-core CTA streams at most when it groups partitions:
-// 1024 over 16-bit caches, 4096 over FP8 ones, whose chunks take half the
-// time and so pay relatively twice the per-CTA cost.
-int tc_group_blocks(bool fp8) { return fp8 ? 256 : 64; }
+// 2048 over 16-bit caches, 4096 over FP8 ones, whose chunks take half the
+// time and so pay relatively twice the per-CTA cost (measured at the 70B
+// shape's 512-token partitions: 184.4 us grouped to 2048 against 188.8 at
+// 1024; over FP8 116.3 us grouped to 4096).
+int tc_group_blocks(bool fp8) { return fp8 ? 256 : 128; }
 
 // Partitions one tensor-core CTA streams back to back: partitions shorter
 // than the group size that start on a chunk are grouped up to it per CTA,
@@ -143,15 +145,17 @@ int tc_heads_per_cta(const Plan &pl, const pa_dims *d, int rows, bool plain) {
 }
 
 // Automatic partition of the tensor-core kernel: the largest of 4096 (FP8
-// caches only), 2048 and 1024 tokens at which the batch still gives two
-// waves of resident CTAs.  A CTA pays its set-up, first loads and drain
-// once per partition, and over an FP8 cache its chunks take half the time
-// (measured on the 8B continuous-batching step: 156 us at 2048 against 159
-// at 1024 over a 16-bit cache; 102 us at 4096, 109 at 2048 and 141 at 1024
-// over an FP8 one).
+// caches, and the 16-row shape that runs two CTAs per SM), 2048 and 1024
+// tokens at which the batch still gives two waves of resident CTAs.  A CTA
+// pays its set-up, first loads and drain once per partition.  Measured: the
+// 8B continuous-batching step 156 us at 2048 against 159 at 1024 and 173 at
+// 4096 over a 16-bit cache, 102 us at 4096, 109 at 2048 and 141 at 1024
+// over an FP8 one; the 8B step with 4 query tokens (16 rows) 260.6 us at
+// 4096 against 267.0 at 2048.
 int tc_auto_partition(const pa_dims *d, int ctx_blocks, int rows, bool fp8) {
     const int64_t pairs = (int64_t)d->num_seqs * d->num_kv_heads;
-    for (int P = fp8 ? 4 * kAutoPartitionTc : 2 * kAutoPartitionTc; P > kAutoPartitionTc; P /= 2) {
+    const bool wide = fp8 || rows > 8;
+    for (int P = wide ? 4 * kAutoPartitionTc : 2 * kAutoPartitionTc; P > kAutoPartitionTc; P /= 2) {
         const int blocks = P / 16;
         if (pairs * ((ctx_blocks + blocks - 1) / blocks) >= 2 * tc_slots(rows, fp8)) return P;
     }

@@ -82,6 +82,8 @@ def test_workspace_plan(lib):
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=f8), 4096, 0) == 1
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, kv_dtype=f8, max_blocks_per_seq=512), 8192, 0) == 2
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=32, kv_dtype=f8, max_blocks_per_seq=512), 8192, 0) == 4
+    # and for 16 query rows per KV head (two CTAs per SM)
+    assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, num_heads=128), 4096, 0) == 1
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=16), 4096, 0) == 4  # 256 CTAs at 2048: 1024
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, num_heads=8), 4096, 0) == 8  # CUDA-core: 512
 
