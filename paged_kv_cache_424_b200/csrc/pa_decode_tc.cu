@@ -326,7 +326,10 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     const int H = p.num_heads, head0 = kvh * G;  // head0: unmasked launches (group == G, q_len == 1)
     T *out = reinterpret_cast<T *>(p.out);
     pdl_launch_dependents();
-    pdl_wait();
+    // Until pdl_wait() below the CTA reads only inputs that no kernel of this
+    // library writes (seq_order, block table, context length, q), so this
+    // part overlaps the tail of the kernel before it on the stream; the
+    // caches, the output and the workspace are touched after the wait.
     const int s = scheduled_seq(p, g_seq, part0 == 0 && g_head == 0 && tid == 0);
     if (s < 0) return;
     // Without a window a CTA's slice of the table starts at part0 *
@@ -353,6 +356,33 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     if (part0 >= nparts) return;
     const int nmine = min(ppc, nparts - part0);  // partitions of this CTA
     const bool direct = nparts == 1;
+    // The softmax warps load their query rows now, before the set-up: E4M3,
+    // a warp per row (rows warp, warp + kSW, ..), 4 dims per lane; 16-bit,
+    // 16-byte pieces (piece i: row i / 16, dims 8 (i % 16) ..)
+    constexpr int kQRowsW = kE4m3 ? (G + kSW - 1) / kSW : 1;
+    constexpr int kQPieces = kE4m3 ? 1 : (kN * (kD / 8) + kST - 1) / kST;
+    uint2 q8[kQRowsW];
+    uint4 q16[kQPieces];
+    if (warp < kSW) {
+        const T *q = reinterpret_cast<const T *>(p.q);
+        if constexpr (kE4m3) {
+#pragma unroll
+            for (int k = 0; k < kQRowsW; ++k) {
+                const int r = warp + k * kSW;
+                q8[k] = r < G && r < rows ? *reinterpret_cast<const uint2 *>(q + row_of(r) * kD + 4 * lane)
+                                          : make_uint2(0, 0);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kQPieces; ++k) {
+                const int i = tid + k * kST, r = i / (kD / 8);
+                q16[k] = i < kN * (kD / 8) && r < rows
+                             ? *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + (i % (kD / 8)) * 8)
+                             : make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    pdl_wait();
     if (L == 0) {
         for (int i = tid; i < rows * kD; i += blockDim.x) out[row_of(i / kD) * kD + i % kD] = E::from_float(0.f);
         return;
@@ -365,15 +395,14 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     const int b0 = sp.bfirst + part0 * p.part_blocks;
     const int nb = min(nmine * p.part_blocks, nblk - b0);  // blocks of this CTA's partitions
     const int nch = (nb + kChunkBlocks - 1) / kChunkBlocks; // chunks of 128 tokens
-    // chunks per partition: partitions of several chunks start on a chunk
-    // (the host sets ppc > 1 only when part_blocks is a multiple of 8)
-    // One partial per CTA: the partitions a CTA streams are combined into
-    // the slot of its first one, and the others are marked empty (lse =
-    // -inf, weight 0 in the merge), so the pipeline runs through partition
-    // boundaries instead of draining at each (chunks per written partial).
+    // One partial per CTA: the partitions a CTA streams (ppc > 1 only when
+    // they start on a chunk) are combined into the slot of its first one,
+    // and the others are marked empty (lse = -inf, weight 0 in the merge),
+    // so the pipeline runs through partition boundaries instead of draining
+    // at each.  cpp: chunks per written partial, all of a head's chunks.
     const int cpp = nch;
     const int tok0 = b0 * kBlock;
-    const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this partition: [tok0, tok_end)
+    const int tok_end = min(L, (b0 + nb) * kBlock);         // tokens of this CTA: [tok0, tok_end)
     const int nct = hpc * nch;                              // chunks of all the CTA's heads
 
     // ---- set-up -----------------------------------------------------------------
@@ -507,8 +536,8 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
     } else if (warp < kSW) {
         // ------------------------------ softmax warps ------------------------------
         {
-            // Q tile, loaded while the producers already stream K and V.
-            const T *q = reinterpret_cast<const T *>(p.q);
+            // Q tile (rows loaded before the set-up), written while the
+            // producers already stream K and V.
             if constexpr (kE4m3) {
                 // Q as E4M3 parts, one warp per query row r, lane l holding
                 // dims 4l .. 4l + 3: y = q * 2^e with max |y| in [128, 256),
@@ -516,11 +545,13 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
                 // so q = 2^-e (hi + mid / 16 + lo / 256) + err, |err| <= 2^-15 max |q|.
                 // Rows hi: r, mid: G + r, lo: 2G + r of the 128-byte-swizzled
                 // tile; padding rows zero.  qscale[r] = scale_log2 * 2^-e.
-                for (int r = warp; r < G; r += kSW) {
-                    float y[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (r < rows) {
-                        const uint2 raw = *reinterpret_cast<const uint2 *>(q + row_of(r) * kD + 4 * lane);
-                        const float2 a = E::to_float2(raw.x), b = E::to_float2(raw.y);
+#pragma unroll
+                for (int kr = 0; kr < kQRowsW; ++kr) {
+                    const int r = warp + kr * kSW;
+                    if (r >= G) break;  // warp-uniform
+                    float y[4];
+                    {
+                        const float2 a = E::to_float2(q8[kr].x), b = E::to_float2(q8[kr].y);  // 0 past rows
                         y[0] = a.x;
                         y[1] = a.y;
                         y[2] = b.x;
@@ -556,11 +587,13 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
             } else {
                 // rows = the group's query heads (zero rows up to 16), K-major
                 // 128-byte swizzle, two 64-dim regions
-                for (int i = tid; i < kN * (kD / 8); i += kST) {
+#pragma unroll
+                for (int k = 0; k < kQPieces; ++k) {
+                    const int i = tid + k * kST;
+                    if (i >= kN * (kD / 8)) break;
                     const int r = i / (kD / 8), c16 = i % (kD / 8);  // row, 16-byte chunk
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (r < rows) v = *reinterpret_cast<const uint4 *>(q + row_of(r) * kD + c16 * 8);
-                    *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) = v;
+                    *reinterpret_cast<uint4 *>(q_t + (c16 >> 3) * (kN * 128) + tc::sw128_offset(r, (c16 & 7) * 8)) =
+                        q16[k];
                 }
             }
             fence_proxy_async_smem();
@@ -638,7 +671,7 @@ __global__ void __launch_bounds__(tc_threads(G, kFp8), tc_ctas_per_sm(G, kFp8))
             if (wait_o(c)) load_o(c, hgc);
         };
         const bool has_tail = (b0 + nb == nblk) && (L % kBlock) != 0;  // partial last block here
-        // the partial of partition part0 + pi of head kvh + hh: per-column
+        // the partial (pi = 0, in partition part0's slot) of head kvh + hh: per-column
         // sums over the 4 lane quadrants, then o = acc / l (and lse) to the
         // output or the workspace; the last sync frees `red` for the next
         // chunk's maxima (fewer syncs made the compiler spill in the loop)
