@@ -28,12 +28,13 @@ pa_status cuda_fail(cudaError_t e, const char *what) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Automatic partition size, measured on B200: 512 tokens for the CUDA-core
-// kernel (its per-warp rings favour many short items), 1024 tokens (8 chunks
-// of 128) for the tensor-core kernel, whose per-CTA set-up (TMEM, barriers,
-// Q tile) then amortises over more chunks while long contexts still give
-// thousands of CTAs.  The merge costs ~1-2% of the KV traffic either way.
+// kernel (its per-warp rings favour many short items); for the tensor-core
+// kernel at least 1024 tokens (8 chunks of 128), whose per-CTA set-up
+// (TMEM, barriers, Q tile) then amortises over more chunks, and more for
+// batches large enough (tc_auto_partition).  The merge costs ~1-2% of the
+// KV traffic either way.
 constexpr int kAutoPartitionSimt = 512;
-constexpr int kAutoPartitionTc = 1024;  // up to 4x for large batches (tc_auto_partition)
+constexpr int kAutoPartitionTc = 1024;
 constexpr int kMaxPartitionTokens = 32768;
 
 bool kv_fp8(const pa_dims *d) { return d->kv_dtype == PA_FP8_E4M3; }

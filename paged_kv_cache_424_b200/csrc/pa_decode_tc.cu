@@ -9,8 +9,10 @@
 //   O^T (128 dims x 16)  = V^T (128 x 128 tokens) . P^T (128 x 16)  [PV]
 // (the G query rows padded to the MMA's N = 16).
 //
-// CTA = (partition, KV head, sequence): 8 warps (12 with 16 columns, whose
-// softmax work is split over 8 warps, 8 columns each); the last warp idles.
+// CTA = (partition, KV head, sequence), or a group of consecutive
+// partitions or of two KV heads (set by the host): 8 warps (12 with 16
+// columns, whose softmax work is split over 8 warps, 8 columns each); the
+// last warp idles.
 //   warp 4  K producer and warp 6  V producer (8 and 10 with 16 columns): per chunk, 2-D tiled TMA loads
 //           of the 8 blocks' K (or V) rows (16 rows x 64 dims per box,
 //           128-byte swizzle) into the K (or V) tile, as soon as the previous
