@@ -88,6 +88,37 @@ def test_workspace_plan(lib):
     assert lib.pa_decode_num_partitions(_dims(lib, num_seqs=256, num_heads=8), 4096, 0) == 8  # CUDA-core: 512
 
 
+def test_plan_is_consistent_over_random_shapes(lib):
+    """For random batches, lengths, groups, cache types and partition
+    sizes: the workspace is zero exactly when the plan has one partition,
+    and otherwise holds an fp32 row of head_dim values and an lse for every
+    (query row, partition); automatic partitions never split the longest
+    context into more pieces than 1024-token ones would (512-token ones on
+    the CUDA-core kernel)."""
+    import numpy as np
+    rng = np.random.default_rng(2024)
+    for _ in range(400):
+        g = int(rng.choice([1, 2, 4, 8, 16]))
+        hk = int(rng.choice([1, 2, 4, 8]))
+        d = int(rng.choice([64, 128]))
+        mb = int(rng.integers(1, 600))
+        kv = int(rng.choice([0, lib.PA_FP8_E4M3]))
+        dims = _dims(lib, num_seqs=int(rng.integers(1, 600)), num_heads=g * hk, num_kv_heads=hk, head_dim=d,
+                     max_blocks_per_seq=mb, kv_dtype=kv)
+        maxlen = int(rng.integers(0, mb * 16 + 1))
+        P = int(rng.choice([0, 0, 16, 128, 512, 1024, 4096]))
+        parts = lib.pa_decode_num_partitions(dims, maxlen, P)
+        ws = lib.pa_decode_workspace_size(dims, maxlen, P)
+        assert parts >= 1
+        if parts == 1:
+            assert ws == 0
+        else:
+            rows = dims.num_seqs * dims.num_heads * parts
+            assert ws >= rows * d * 4 + rows * 4
+        if P == 0 and maxlen > 0:
+            assert parts <= -(-maxlen // 512) if (g < 4 or d != 128) else parts <= -(-maxlen // 1024)
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(block_size=32), -4), (dict(head_dim=96), -4), (dict(num_heads=24, num_kv_heads=8), -4),
     (dict(num_heads=30), -3), (dict(dtype=7), -2), (dict(num_kv_heads=0), -3), (dict(num_seqs=-1), -3),
